@@ -1,0 +1,124 @@
+"""float64 CPU oracle for sliding-window causal attention.
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the benchmark's
+CPU-baseline leg may import this package. The CUDA library never imports it, shares
+no code with it and never falls back to it.
+
+What it computes is written out in swa_oracle.c (plain float64 loops, OpenMP over
+rows). This module only marshals numpy arrays into that library with ctypes.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load(path=None):
+    global _lib
+    if path is not None:
+        lib = ctypes.CDLL(path)
+    else:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(_build.build())
+    d = ctypes.POINTER(ctypes.c_double)
+    i64 = ctypes.c_int64
+    pi64 = ctypes.POINTER(ctypes.c_int64)
+    lib.swa_oracle_forward.argtypes = [d, d, d, d, i64, i64, i64, i64, i64]
+    lib.swa_oracle_forward_rows.argtypes = [d, d, d, i64, i64, i64, i64, i64, pi64, i64, d]
+    lib.swa_oracle_weights.argtypes = [d, d, d, i64, i64, i64, i64, i64]
+    lib.swa_oracle_decode.argtypes = [d, d, d, pi64, d, i64, i64, i64, i64]
+    for f in (lib.swa_oracle_forward, lib.swa_oracle_forward_rows, lib.swa_oracle_weights,
+              lib.swa_oracle_decode):
+        f.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _f64(a):
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _i64(a):
+    a = np.ascontiguousarray(a, dtype=np.int64)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+class OracleError(ValueError):
+    pass
+
+
+def forward(q, k, v, W, lib=None):
+    """out[B,H,T,D] (float64) for q, k, v of shape [B,H,T,D] and window W."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    k, pk = _f64(k)
+    v, pv = _f64(v)
+    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise OracleError("q, k, v must share one [B,H,T,D] shape")
+    B, H, T, D = q.shape
+    out = np.empty_like(q)
+    _, po = _f64(out)
+    rc = lib.swa_oracle_forward(pq, pk, pv, po, B, H, T, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle forward rejected its arguments (rc={rc})")
+    return out
+
+
+def forward_rows(q, k, v, W, rows, lib=None):
+    """Outputs [n, D] of the flattened query rows r = (b*H + h)*T + i listed in rows."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    k, pk = _f64(k)
+    v, pv = _f64(v)
+    B, H, T, D = q.shape
+    rows, pr = _i64(rows)
+    out = np.empty((rows.shape[0], D), dtype=np.float64)
+    _, po = _f64(out)
+    rc = lib.swa_oracle_forward_rows(pq, pk, pv, B, H, T, D, int(W), pr, rows.shape[0], po)
+    if rc != 0:
+        raise OracleError(f"oracle forward_rows rejected its arguments (rc={rc})")
+    return out
+
+
+def weights(q, k, W, lib=None):
+    """Attention weights [B,H,T,T] of the definition (small inputs only)."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    k, pk = _f64(k)
+    B, H, T, D = q.shape
+    w = np.empty((B, H, T, T), dtype=np.float64)
+    _, pw = _f64(w)
+    rc = lib.swa_oracle_weights(pq, pk, pw, B, H, T, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle weights rejected its arguments (rc={rc})")
+    return w
+
+
+def decode(q, kring, vring, pos, W, lib=None):
+    """out[B,H,D] for one query per stream over the rolling buffer (slot = pos mod W)."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    kring, pk = _f64(kring)
+    vring, pv = _f64(vring)
+    pos, pp = _i64(pos)
+    B, H, D = q.shape
+    if kring.shape != (B, H, W, D) or vring.shape != (B, H, W, D) or pos.shape != (B,):
+        raise OracleError("rings must be [B,H,W,D] and pos [B]")
+    out = np.empty_like(q)
+    _, po = _f64(out)
+    rc = lib.swa_oracle_decode(pq, pk, pv, pp, po, B, H, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle decode rejected its arguments (rc={rc})")
+    return out
+
+
+def load_variant(path):
+    """Load another build of swa_oracle.c (used by the mutation tests)."""
+    return _load(path)

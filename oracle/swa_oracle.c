@@ -1,0 +1,240 @@
+/*
+ * swa_oracle.c: float64 CPU oracle for sliding-window causal attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this code. It shares no source, header,
+ * helper or constant with the CUDA library, and the CUDA library never calls it.
+ *
+ * What it computes: the plain definition, written out with no blocking, fusion
+ * or reordering. For every batch b, head h and query position i:
+ *
+ *   band(i) = { j : max(0, i-W+1) <= j <= i }
+ *       "27. Sliding-Window Attention", Step-by-Step Approach, step 2: the band
+ *       mask is (j <= i) & (i - j < window_size).
+ *       "25. Sliding-Window Causal Attention for Streaming Inference",
+ *       Step-by-Step Approach, step 3: key_pos <= query_pos and
+ *       key_pos > query_pos - window_size.
+ *       "NNX Sliding-Window Attention", opening paragraph: keys from
+ *       max(0, i - W + 1) through i.
+ *   s_j    = (sum_d q[b,h,i,d] * k[b,h,j,d]) / sqrt(D)       for j in band(i)
+ *       "27. Sliding-Window Attention", Step-by-Step Approach, step 1.
+ *   m      = max_j s_j
+ *   e_j    = exp(s_j - m)
+ *       "Mistral Architecture > Implementation: Sliding Window Attention",
+ *       Step 2 (stable softmax: subtract the row maximum before exponentiating).
+ *   out[b,h,i,:] = (sum_j e_j * v[b,h,j,:]) / (sum_j e_j)
+ *       "27. Sliding-Window Attention", Step-by-Step Approach, step 5
+ *       (softmax over the keys, then weights @ v).
+ *
+ * Keys outside band(i) are never read: a masked score has exactly zero weight
+ * after the softmax, so leaving it out of the sums is the same result
+ * ("27. Sliding-Window Attention", step 3). The loops run in plain order:
+ * j ascending, d ascending. All arithmetic is IEEE float64. There is no -ffast-math.
+ *
+ * Layout: every tensor is row-major contiguous [B, H, T, D], so element
+ * (b,h,t,d) sits at ((b*H + h)*T + t)*D + d ("27. Sliding-Window Attention",
+ * reference solution: q has shape (batch, heads, seq, head_dim)).
+ *
+ * Decode: the rolling buffer keeps the last W positions of each stream. Position
+ * p lives in slot p mod W ("25. Sliding-Window Causal Attention for Streaming
+ * Inference", Problem: a bounded KV cache that evicts anything older than the
+ * window). For stream b at absolute position P the query attends to positions
+ * max(0, P-W+1) .. P, in ascending position order, read from slot p mod W.
+ *
+ * Return codes: 0 on success, 1 for an invalid argument (W < 1, a negative size,
+ * a null pointer, a negative position). On error nothing is written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_INVALID 1
+
+/* One query row of the prefill definition. qi: [D]. kh, vh: [T, D] for one (b,h).
+ * out: [D]. scores: scratch of at least min(i+1, W) doubles. */
+static void oracle_row(const double* qi, const double* kh, const double* vh,
+                       int64_t i, int64_t D, int64_t W, double* scores, double* out) {
+    int64_t lo = i - W + 1;
+    if (lo < 0) lo = 0;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+
+    /* scores over the band, j ascending */
+    double m = -INFINITY;
+    for (int64_t j = lo; j <= i; ++j) {
+        const double* kj = kh + j * D;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qi[d] * kj[d];
+        double s = dot * inv_sqrt_d;
+        scores[j - lo] = s;
+        if (s > m) m = s;
+    }
+
+    /* e_j = exp(s_j - m); numerator and denominator, j ascending */
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    double denom = 0.0;
+    for (int64_t j = lo; j <= i; ++j) {
+        double e = exp(scores[j - lo] - m);
+        denom += e;
+        const double* vj = vh + j * D;
+        for (int64_t d = 0; d < D; ++d) out[d] += e * vj[d];
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] = out[d] / denom;
+}
+
+static int check_sizes(int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (W < 1 || B < 0 || H < 0 || T < 0 || D < 1) return ORACLE_INVALID;
+    return ORACLE_OK;
+}
+
+/* Full prefill: out[B,H,T,D] for every row. */
+int swa_oracle_forward(const double* q, const double* k, const double* v, double* out,
+                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK) return ORACLE_INVALID;
+    if (B * H * T == 0) return ORACLE_OK;
+    if (!q || !k || !v || !out) return ORACLE_INVALID;
+    const int64_t nrows = B * H * T;
+    const int64_t band_max = (W < T) ? W : T;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* scores = (double*)malloc((size_t)band_max * sizeof(double));
+        if (!scores) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 64)
+            for (int64_t r = 0; r < nrows; ++r) {
+                const int64_t bh = r / T, i = r % T;
+                const double* kh = k + bh * T * D;
+                const double* vh = v + bh * T * D;
+                oracle_row(q + r * D, kh, vh, i, D, W, scores, out + r * D);
+            }
+            free(scores);
+        }
+    }
+    return bad ? ORACLE_INVALID : ORACLE_OK;
+}
+
+/* Selected rows only: rows[n] holds flattened row indices r = (b*H + h)*T + i.
+ * out_rows: [n, D], row t of it is the output of query row rows[t]. */
+int swa_oracle_forward_rows(const double* q, const double* k, const double* v,
+                            int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                            const int64_t* rows, int64_t n, double* out_rows) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK || n < 0) return ORACLE_INVALID;
+    if (n == 0) return ORACLE_OK;
+    if (!q || !k || !v || !rows || !out_rows) return ORACLE_INVALID;
+    for (int64_t t = 0; t < n; ++t)
+        if (rows[t] < 0 || rows[t] >= B * H * T) return ORACLE_INVALID;
+    const int64_t band_max = (W < T) ? W : T;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* scores = (double*)malloc((size_t)band_max * sizeof(double));
+        if (!scores) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < n; ++t) {
+                const int64_t r = rows[t];
+                const int64_t bh = r / T, i = r % T;
+                oracle_row(q + r * D, k + bh * T * D, v + bh * T * D, i, D, W, scores,
+                           out_rows + t * D);
+            }
+            free(scores);
+        }
+    }
+    return bad ? ORACLE_INVALID : ORACLE_OK;
+}
+
+/* Attention weights of the definition, for checking probabilities on small
+ * inputs: weights[B,H,T,T], zero outside the band, e_j / sum e_j inside. */
+int swa_oracle_weights(const double* q, const double* k, double* weights,
+                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK) return ORACLE_INVALID;
+    if (B * H * T == 0) return ORACLE_OK;
+    if (!q || !k || !weights) return ORACLE_INVALID;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        for (int64_t i = 0; i < T; ++i) {
+            double* wrow = weights + (bh * T + i) * T;
+            for (int64_t j = 0; j < T; ++j) wrow[j] = 0.0;
+            int64_t lo = i - W + 1;
+            if (lo < 0) lo = 0;
+            const double* qi = q + (bh * T + i) * D;
+            double m = -INFINITY;
+            for (int64_t j = lo; j <= i; ++j) {
+                const double* kj = k + (bh * T + j) * D;
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d) dot += qi[d] * kj[d];
+                wrow[j] = dot * inv_sqrt_d;
+                if (wrow[j] > m) m = wrow[j];
+            }
+            double denom = 0.0;
+            for (int64_t j = lo; j <= i; ++j) {
+                wrow[j] = exp(wrow[j] - m);
+                denom += wrow[j];
+            }
+            for (int64_t j = lo; j <= i; ++j) wrow[j] = wrow[j] / denom;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Decode over a rolling buffer. q: [B,H,D]; kring, vring: [B,H,W,D]; pos: [B];
+ * out: [B,H,D]. Stream b attends to positions max(0, P-W+1)..P (P = pos[b]),
+ * ascending, each read from slot p mod W; the same formula as a prefill row. */
+static void oracle_decode_one(const double* qv, const double* kr, const double* vr,
+                              int64_t P, int64_t D, int64_t W, double* scores, double* out) {
+    int64_t first = P - W + 1;
+    if (first < 0) first = 0;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double m = -INFINITY;
+    for (int64_t p = first; p <= P; ++p) {
+        const double* kp = kr + (p % W) * D;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qv[d] * kp[d];
+        double s = dot * inv_sqrt_d;
+        scores[p - first] = s;
+        if (s > m) m = s;
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    double denom = 0.0;
+    for (int64_t p = first; p <= P; ++p) {
+        double e = exp(scores[p - first] - m);
+        denom += e;
+        const double* vp = vr + (p % W) * D;
+        for (int64_t d = 0; d < D; ++d) out[d] += e * vp[d];
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] = out[d] / denom;
+}
+
+int swa_oracle_decode(const double* q, const double* kring, const double* vring,
+                      const int64_t* pos, double* out,
+                      int64_t B, int64_t H, int64_t D, int64_t W) {
+    if (W < 1 || B < 0 || H < 0 || D < 1) return ORACLE_INVALID;
+    if (B * H == 0) return ORACLE_OK;
+    if (!q || !kring || !vring || !pos || !out) return ORACLE_INVALID;
+    for (int64_t b = 0; b < B; ++b)
+        if (pos[b] < 0) return ORACLE_INVALID;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* scores = (double*)malloc((size_t)W * sizeof(double));
+        if (!scores) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bh = 0; bh < B * H; ++bh) {
+                const int64_t b = bh / H;
+                oracle_decode_one(q + bh * D, kring + bh * W * D, vring + bh * W * D,
+                                  pos[b], D, W, scores, out + bh * D);
+            }
+            free(scores);
+        }
+    }
+    return bad ? ORACLE_INVALID : ORACLE_OK;
+}

@@ -1,0 +1,224 @@
+"""Pins that tie the float64 oracle to what the pages and the mathematics fix.
+
+Each pin takes an oracle library handle so that the same checks can run against
+deliberately broken builds of the oracle (tests/test_oracle_mutants.py): every
+plausible mistake there must make at least one pin fail.
+
+None of these pins re-types the oracle's formula. They compare it with printed
+values, with torch's own scaled-dot-product attention (a library routine), with
+a dense masked computation built a different way, with closed forms, and with
+invariants.
+"""
+import numpy as np
+import torch
+
+import oracle
+from oracle import brute
+
+from golden import read_band, read_moving_average
+
+TIGHT = 1e-12
+
+
+def _sdpa(q, k, v, mask=None, causal=False):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    out = torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=None if mask is None else torch.from_numpy(mask),
+        dropout_p=0.0, is_causal=causal)
+    return out.numpy()
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def pin_band_masks(lib):
+    """q = k = 0 and v = identity (D = T) make output row i equal to
+    1/|band(i)| on the band's columns and 0 elsewhere, so the oracle's own band
+    can be read off its output. It must equal the two printed masks bit for bit,
+    and the brute-force pair enumeration for every small (T, W)."""
+    def oracle_band(T, W):
+        q = np.zeros((1, 1, T, T))
+        v = np.eye(T).reshape(1, 1, T, T)
+        out = oracle.forward(q, q, v, W, lib=lib)[0, 0]
+        mask = out > 0
+        counts = mask.sum(axis=1)
+        # within the band every weight is exactly 1/count (exp(0) = 1, exact division)
+        assert np.array_equal(out[mask], np.repeat(1.0 / counts, counts)), "band weights"
+        return mask
+
+    for name in ("nnx_band_T5_W3.txt", "mistral_impl_band_T8_W4.txt"):
+        T, W, printed = read_band(name)
+        assert np.array_equal(oracle_band(T, W), printed), f"printed mask {name}"
+    for T in (1, 2, 3, 7, 16, 33):
+        for W in (1, 2, 3, 5, 8, 15, 16, 17, 40):
+            m = oracle_band(T, W)
+            assert np.array_equal(m, brute.band_mask(T, W)), f"band T={T} W={W}"
+            assert np.array_equal(m.sum(axis=1), np.minimum(np.arange(T) + 1, W))
+
+
+def pin_moving_average(lib):
+    """The worked example with zero q/k projections prints exact trailing means,
+    and changing input row 0 leaves rows 3 and later unchanged."""
+    g = read_moving_average()
+    W, x = g["W"], g["x"]
+    T, Hn = x.shape
+    v = x.T.reshape(1, Hn, T, 1).copy()
+    z = np.zeros_like(v)
+    out = oracle.forward(z, z, v, W, lib=lib)[0, :, :, 0].T
+    assert np.array_equal(out, g["y"]), "moving average printed values"
+    row, vals = g["changed_row"]
+    x2 = x.copy()
+    x2[row] = vals
+    v2 = x2.T.reshape(1, Hn, T, 1).copy()
+    out2 = oracle.forward(z, z, v2, W, lib=lib)[0, :, :, 0].T
+    u = g["unchanged_from"]
+    assert np.array_equal(out2[u:], out[u:]), "rows past the window unchanged"
+    assert not np.array_equal(out2[:u], out[:u])
+
+
+def pin_trailing_mean_any_k(lib):
+    """Generalisation of the worked example: q = 0 gives the trailing mean of v over
+    the band whatever k holds (every score is 0, so all weights are equal)."""
+    rng = np.random.default_rng(7)
+    for (T, D, W) in ((9, 3, 4), (20, 5, 1), (12, 2, 30)):
+        q = np.zeros((1, 2, T, D))
+        k = _rand(rng, 1, 2, T, D)
+        v = _rand(rng, 1, 2, T, D)
+        out = oracle.forward(q, k, v, W, lib=lib)
+        for i in range(T):
+            lo = max(0, i - W + 1)
+            ref = v[:, :, lo:i + 1, :].mean(axis=2)
+            assert np.abs(out[:, :, i, :] - ref).max() <= TIGHT, "trailing mean"
+
+
+def pin_causal_reduction(lib):
+    """W >= T is ordinary causal attention: compare with torch's scaled dot-product
+    attention (is_causal=True) in float64."""
+    rng = np.random.default_rng(11)
+    for (B, H, T, D) in ((1, 2, 6, 4), (2, 3, 17, 8), (1, 1, 40, 1)):
+        q, k, v = (_rand(rng, B, H, T, D) for _ in range(3))
+        ref = _sdpa(q, k, v, causal=True)
+        for W in (T, T + 1, 3 * T):
+            out = oracle.forward(q, k, v, W, lib=lib)
+            assert np.abs(out - ref).max() <= TIGHT, f"causal W={W}"
+
+
+def pin_general_band(lib):
+    """Random inputs, general W: compare with torch's scaled dot-product attention
+    given the brute-force boolean band mask, and with the dense masked computation."""
+    rng = np.random.default_rng(13)
+    for (B, H, T, D, W) in ((1, 2, 6, 4, 3), (2, 2, 19, 5, 4), (1, 3, 33, 16, 7),
+                            (1, 1, 12, 2, 11), (1, 2, 25, 3, 2)):
+        q, k, v = (_rand(rng, B, H, T, D) * 2.0 for _ in range(3))
+        out = oracle.forward(q, k, v, W, lib=lib)
+        ref = _sdpa(q, k, v, mask=brute.band_mask(T, W))
+        assert np.abs(out - ref).max() <= TIGHT, f"sdpa band T={T} W={W}"
+        ref2, _ = brute.dense_masked_attention(q, k, v, W)
+        assert np.abs(out - ref2).max() <= TIGHT, f"dense band T={T} W={W}"
+
+
+def pin_window_one(lib):
+    """W = 1 keeps only the diagonal, so the output is v exactly."""
+    rng = np.random.default_rng(17)
+    q, k, v = (_rand(rng, 2, 3, 10, 6) for _ in range(3))
+    assert np.array_equal(oracle.forward(q, k, v, 1, lib=lib), v), "W=1 returns v"
+
+
+def pin_independence(lib):
+    """Corrupt-and-compare: changing k and v at positions j <= i - W leaves row i
+    unchanged exactly; changing a position inside the window changes it."""
+    rng = np.random.default_rng(19)
+    B, H, T, D, W = 1, 2, 24, 4, 5
+    q, k, v = (_rand(rng, B, H, T, D) for _ in range(3))
+    base = oracle.forward(q, k, v, W, lib=lib)
+    for i in (W, 11, T - 1):
+        k2, v2 = k.copy(), v.copy()
+        k2[:, :, : i - W + 1, :] = 100.0
+        v2[:, :, : i - W + 1, :] = 200.0
+        out = oracle.forward(q, k2, v2, W, lib=lib)
+        assert np.array_equal(out[:, :, i, :], base[:, :, i, :]), f"row {i} independent"
+        k3 = k.copy()
+        k3[:, :, i - W + 1, :] += 1.0
+        out3 = oracle.forward(q, k3, v, W, lib=lib)
+        assert not np.array_equal(out3[:, :, i, :], base[:, :, i, :]), f"row {i} sees j=i-W+1"
+
+
+def pin_weights(lib):
+    """Probabilities: zero outside the band, each row sums to 1, weights @ v is the output."""
+    rng = np.random.default_rng(23)
+    B, H, T, D, W = 1, 2, 16, 32, 4
+    q, k, v = (_rand(rng, B, H, T, D) for _ in range(3))
+    w = oracle.weights(q, k, W, lib=lib)
+    mask = brute.band_mask(T, W)
+    assert np.all(w[:, :, ~mask] == 0.0), "off-band weights are zero"
+    assert np.all(w[:, :, mask] > 0.0)
+    assert np.abs(w.sum(axis=-1) - 1.0).max() <= TIGHT, "rows sum to 1"
+    out = oracle.forward(q, k, v, W, lib=lib)
+    assert np.abs(np.matmul(w, v) - out).max() <= TIGHT
+    _, wref = brute.dense_masked_attention(q, k, v, W)
+    assert np.abs(w - wref).max() <= TIGHT
+
+
+def pin_rows_subset(lib):
+    """forward_rows returns exactly the rows of the full forward."""
+    rng = np.random.default_rng(29)
+    B, H, T, D, W = 2, 2, 21, 5, 6
+    q, k, v = (_rand(rng, B, H, T, D) for _ in range(3))
+    full = oracle.forward(q, k, v, W, lib=lib).reshape(-1, D)
+    rows = np.array([0, 5, 20, 21, 40, 63, B * H * T - 1])
+    sub = oracle.forward_rows(q, k, v, W, rows, lib=lib)
+    assert np.array_equal(sub, full[rows])
+
+
+def _ring_from_history(kh, vh, P, W):
+    """Write positions 0..P of a history [P+1, D] into a W-slot ring, slot p mod W,
+    later positions overwriting earlier ones (brute force, position by position)."""
+    D = kh.shape[-1]
+    kr = np.zeros((W, D))
+    vr = np.zeros((W, D))
+    for p in range(P + 1):
+        kr[p % W] = kh[p]
+        vr[p % W] = vh[p]
+    return kr, vr
+
+
+def pin_decode(lib):
+    """Decode over a ring built from a seeded history equals the last row of the
+    prefill over that history; for P >= W-1 the answer depends only on the ring."""
+    rng = np.random.default_rng(31)
+    D, H = 6, 2
+    for W in (1, 3, 8):
+        for P in sorted({0, 1, max(0, W - 2), W - 1, W, W + 1, 2 * W + 3, 3 * W}):
+            B = 2
+            kh = _rand(rng, B, H, P + 1, D)
+            vh = _rand(rng, B, H, P + 1, D)
+            qh = _rand(rng, B, H, P + 1, D)
+            kr = np.zeros((B, H, W, D))
+            vr = np.zeros((B, H, W, D))
+            for b in range(B):
+                for h in range(H):
+                    kr[b, h], vr[b, h] = _ring_from_history(kh[b, h], vh[b, h], P, W)
+            pos = np.array([P, P])
+            out = oracle.decode(qh[:, :, P, :], kr, vr, pos, W, lib=lib)
+            ref = oracle.forward(qh, kh, vh, W, lib=lib)[:, :, P, :]
+            assert np.abs(out - ref).max() <= TIGHT, f"decode W={W} P={P}"
+            if P >= W - 1:
+                out2 = oracle.decode(qh[:, :, P, :], kr, vr, pos + 3 * W, W, lib=lib)
+                assert np.abs(out2 - out).max() <= TIGHT, "full ring independent of P"
+
+
+def pin_shapes(lib):
+    """Printed shapes: (1,2,6,4) with window 3 keeps its shape; the 3-D (1,5,3)
+    case with window 2 is one head."""
+    rng = np.random.default_rng(37)
+    q = _rand(rng, 1, 2, 6, 4)
+    assert oracle.forward(q, q, q, 3, lib=lib).shape == (1, 2, 6, 4)
+    q3 = _rand(rng, 1, 5, 3)
+    out = oracle.forward(q3[:, None], q3[:, None], q3[:, None], 2, lib=lib)[:, 0]
+    assert out.shape == (1, 5, 3)
+
+
+ALL_PINS = [pin_band_masks, pin_moving_average, pin_trailing_mean_any_k, pin_causal_reduction,
+            pin_general_band, pin_window_one, pin_independence, pin_weights, pin_rows_subset,
+            pin_decode, pin_shapes]

@@ -1,0 +1,77 @@
+"""Mutation check of the pins: each plausible mistake planted in a copy of the oracle's
+C source, on the CPU, must make at least one pin fail.
+
+Each mutant is compiled and checked in a child process, so a mutant that corrupts
+memory cannot take the test session down with it (a crash is reported, not counted
+as caught).
+"""
+import json
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+from oracle import build as obuild
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+
+# The scratch for scores holds min(W, T) entries (W for decode); mutants that visit
+# one more key widen it too, so that they stay in bounds and fail on values alone.
+WIDER_SCRATCH = [("const int64_t band_max = (W < T) ? W : T;", "const int64_t band_max = W + 1;"),
+                 ("malloc((size_t)W * sizeof(double))", "malloc((size_t)(W + 1) * sizeof(double))")]
+
+# (name, list of (text to find, replacement))
+MUTANTS = [
+    ("band one key wider (the [i-W, i] reading)",
+     [("int64_t lo = i - W + 1;", "int64_t lo = i - W;")] + WIDER_SCRATCH),
+    ("band one key narrower", [("int64_t lo = i - W + 1;", "int64_t lo = i - W + 2;")]),
+    ("scale 1/D instead of 1/sqrt(D)", [("1.0 / sqrt((double)D)", "1.0 / (double)D")]),
+    ("no scale", [("double s = dot * inv_sqrt_d;", "double s = dot;")]),
+    ("scores read v instead of k",
+     [("const double* kj = kh + j * D;", "const double* kj = vh + j * D;")]),
+    ("exponent sign flipped", [("exp(scores[j - lo] - m)", "exp(m - scores[j - lo])")]),
+    ("denominator dropped", [("out[d] = out[d] / denom;", "out[d] = out[d];")]),
+    ("value row fixed at the band start",
+     [("const double* vj = vh + j * D;", "const double* vj = vh + lo * D;")]),
+    ("decode wrong slot", [("(p % W) * D", "((p + 1) % W) * D")]),
+    ("decode one extra position",
+     [("int64_t first = P - W + 1;", "int64_t first = P - W;")] + WIDER_SCRATCH),
+    ("weights unnormalised", [("wrow[j] = wrow[j] / denom;", "wrow[j] = wrow[j];")]),
+]
+
+_CHILD = r"""
+import json, sys
+sys.path[:0] = [{root!r}, {here!r}]
+import oracle
+from oracle_pins import ALL_PINS
+lib = oracle.load_variant({so!r})
+failed = []
+for pin in ALL_PINS:
+    try:
+        pin(lib)
+    except AssertionError:
+        failed.append(pin.__name__)
+print(json.dumps(failed))
+"""
+
+
+@pytest.mark.parametrize("name,edits", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, edits):
+    src = open(obuild.SRC).read()
+    for old, new in edits:
+        assert old in src, f"mutation anchor missing: {old}"
+        src = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as d:
+        cpath = os.path.join(d, "mutant.c")
+        with open(cpath, "w") as f:
+            f.write(src)
+        so = obuild.build(src=cpath, out=os.path.join(d, "mutant.so"), force=True)
+        code = _CHILD.format(root=ROOT, here=HERE, so=so)
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                           timeout=300)
+        assert r.returncode == 0, f"mutant child crashed: {r.stderr[-2000:]}"
+        failed = json.loads(r.stdout.strip().splitlines()[-1])
+        assert failed, f"no pin caught mutant: {name}"
