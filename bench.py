@@ -1,0 +1,321 @@
+"""Benchmark: sliding-window causal attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+A step is one swa_forward over the Mistral-shaped workload (B=1, H=32, T=16384,
+D=128, W=4096, bf16), inputs resident in HBM. The same run then times swa_decode over
+the streaming workload (B=64 streams, H=32, D=128, W=4096 ring, positions uniform in
+[0, 100000)) in a second timed region and reports it under "decode". Useful prefill
+FLOPs count the band only: 4*B*H*D*sum_i min(i+1, W). Decode bytes are the K/V slots
+read plus q, out and pos.
+
+Under torchrun each rank runs the same workload on its own GPU (weak scaling, no
+collective on the data path); times are the max over ranks. `--impl reference` times
+the float64 CPU oracle on bounded samples of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sliding_window_causal_b200 import inputs  # noqa: E402
+
+METRIC = "SWA prefill TFLOP/s (band FLOPs, % bf16 TC peak); decode HBM GB/s"
+L2_BYTES = 126 * 2**20
+
+
+def band_flops(B, H, T, D, W):
+    # sum_{i<T} min(i+1, W) = W(W+1)/2 + (T-W)W for T >= W, else T(T+1)/2
+    w = min(W, T)
+    s = w * (w + 1) // 2 + (T - w) * w
+    return 4 * B * H * D * s
+
+
+def decode_bytes(B, H, D, W, pos):
+    n = torch.clamp(pos + 1, max=W).sum().item()
+    return int(n * H * D * 2 * 2 + 2 * B * H * D * 2 + 8 * B)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["bf16_tflops"], d["hbm_gbs"], "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.index = period, index
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def timed(fn, steps, stream, pg, device):
+    """Run fn() `steps` times between a barrier + synchronize on both sides; returns
+    the elapsed device time in ms (CUDA events on `stream`), max over ranks."""
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end)
+    if pg is not None:
+        t = torch.tensor([ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        pg.barrier()
+        ms = t.item()
+    return ms
+
+
+def cpu_baseline_prefill(wl, budget_s, q, k, v):
+    """Time the float64 oracle on whole heads of the workload until ~budget_s of CPU
+    work is done. Returns (TFLOP/s, description, threads)."""
+    import numpy as np
+    import oracle
+    flops = 0
+    rows_done = 0
+    t0 = time.perf_counter()
+    h = 0
+    T, D, W = wl.T, wl.D, wl.W
+    chunk = 2048
+    while time.perf_counter() - t0 < budget_s:
+        r0 = (rows_done % T)
+        rows = np.arange(r0, min(T, r0 + chunk), dtype=np.int64)
+        hh = h % wl.H
+        qh, kh, vh = (t[0:1, hh:hh + 1].to(torch.float64).numpy() for t in (q, k, v))
+        oracle.forward_rows(qh, kh, vh, W, rows)
+        flops += int(sum(4 * D * min(i + 1, W) for i in rows))
+        rows_done += len(rows)
+        if rows_done % T == 0:
+            h += 1
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return flops / dt / 1e12, f"{rows_done} query rows of head(s) 0..{h % wl.H} ({dt:.1f} s)", threads
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the float64 CPU oracle on bounded samples of the prefill workload."""
+    if rank != 0:
+        return
+    wl = inputs.MISTRAL
+    q, k, v = inputs.for_workload(wl)
+    per_step = float(os.environ.get("SWA_REF_STEP_S", "4"))
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(wl, per_step / 4, q, k, v)
+    vals = []
+    t0 = time.perf_counter()
+    desc, threads = "", 1
+    for _ in range(args.steps):
+        val, desc, threads = cpu_baseline_prefill(wl, per_step, q, k, v)
+        vals.append(val)
+    dt = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D, "W": wl.W,
+                   "seed": wl.seed},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local, pg = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+
+    import sliding_window_causal_b200 as swa
+    from sliding_window_causal_b200 import _native
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peak_tf, peak_gbs, peak_kind = load_peaks()
+
+    # ------------------------------------------------------------ prefill
+    wl = inputs.MISTRAL
+    qh, kh, vh = inputs.for_workload(wl)
+    q, k, v = (t.to(device) for t in (qh, kh, vh))
+    out = torch.empty_like(q)
+    F = band_flops(wl.B, wl.H, wl.T, wl.D, wl.W)
+    fwd = lambda: swa.forward(q, k, v, wl.W, out=out)
+    for _ in range(args.warmup):
+        fwd()
+    swa.device_status()
+    dev_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
+    with ClockSampler(dev_index) as clk:
+        ms = timed(fwd, args.steps, stream, pg, device)
+    swa.device_status()
+    ms_step = ms / args.steps
+    value = world * F / (ms_step * 1e-3) / 1e12
+    achieved = F / (ms_step * 1e-3) / 1e12
+
+    # ------------------------------------------------------------ e2e (host buffers)
+    pin = lambda t: t.pin_memory()
+    qp, kp, vp = pin(qh), pin(kh), pin(vh)
+    outp = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+    staging = (q, k, v, out)
+    e2e_fn = lambda: swa.forward_host(qp, kp, vp, wl.W, out=outp, device=device, staging=staging)
+    for _ in range(3):
+        e2e_fn()
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = timed(e2e_fn, e2e_steps, stream, pg, device) / e2e_steps
+    swa.device_status()
+    e2e_value = world * F / (e2e_ms * 1e-3) / 1e12
+    h2d = 3 * qh.numel() * qh.element_size()
+    d2h = outp.numel() * outp.element_size()
+    del qp, kp, vp, outp
+
+    # ------------------------------------------------------------ decode
+    decode_line = None
+    if not args.no_decode:
+        del q, k, v, out, staging
+        torch.cuda.empty_cache()
+        dw = inputs.DECODE
+        dq, dkr, dvr, dpos = inputs.for_workload(dw)
+        nbytes = decode_bytes(dw.B, dw.H, dw.D, dw.W, dpos)
+        dq, dkr, dvr, dpos = (t.to(device) for t in (dq, dkr, dvr, dpos))
+        dout = torch.empty_like(dq)
+        dec = lambda: swa.decode(dq, dkr, dvr, dpos, dw.W, out=dout)
+        for _ in range(args.warmup):
+            dec()
+        swa.device_status()
+        with ClockSampler(dev_index) as dclk:
+            dms = timed(dec, args.steps, stream, pg, device) / args.steps
+        swa.device_status()
+        gbs = nbytes / (dms * 1e-3) / 1e9
+        S, chunk = swa.split_plan(dw.B, dw.H, dw.D, dw.W)
+        decode_line = {
+            "metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": dms,
+            "config": {"workload": dw.name, "B": dw.B, "H": dw.H, "D": dw.D, "W": dw.W,
+                       "pos": "uniform [0, 100000)", "seed": dw.seed, "splits": S, "chunk": chunk,
+                       "l2": "inputs larger than L2 (4.3 GB of rings)"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s",
+                         "frac": gbs / peak_gbs, "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes": nbytes},
+            "clocks": dclk.summary(), "gpu_launches": args.steps,
+        }
+
+    # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, desc, threads = cpu_baseline_prefill(wl, float(os.environ.get("SWA_CPU_BUDGET_S", "15")),
+                                                  qh, kh, vh)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D, "W": wl.W,
+                   "seed": wl.seed, "band_flops": F,
+                   "l2": "inputs larger than L2 (q, k, v 384 MB), no flush"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
+                     "traffic": None, "frac_of_spec_2250": achieved / 2250.0},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+        "decode": decode_line,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/*
+ * swa.h: C ABI of the B200 (sm_100a) sliding-window causal attention library.
+ *
+ * The operation. Query position i of a sequence attends only to key positions j
+ * with 0 <= i - j < W, that is to the W most recent positions including itself:
+ *
+ *   out[b,h,i,:] = sum_{j in band(i)} softmax_j( q[b,h,i,:] . k[b,h,j,:] / sqrt(D) ) v[b,h,j,:]
+ *   band(i)      = { j : max(0, i-W+1) <= j <= i }
+ *
+ * Sources: "27. Sliding-Window Attention" (Problem; Step-by-Step Approach steps 1-5:
+ * scaled scores, the band mask (j <= i) & (i - j < window_size), -inf masking,
+ * softmax over keys, weights @ v); "25. Sliding-Window Causal Attention for
+ * Streaming Inference" (Step-by-Step Approach step 3, the strict lower bound
+ * key_pos > query_pos - window_size); "NNX Sliding-Window Attention" (opening
+ * paragraph: keys max(0, i-W+1) .. i; W = 1 is self-attention only; W >= T is
+ * ordinary causal attention). The one-key-wider interval [i-W, i] of "Sliding
+ * Window Attention" (Mathematical Formulation and Attention Masking) is not
+ * used; a caller who wants it passes W+1.
+ *
+ * Conventions for every call below:
+ *  - Every tensor pointer is a DEVICE pointer to row-major contiguous memory, owned
+ *    by the caller. The library keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Calls enqueue work on it and return without waiting (asynchronous).
+ *  - Calls return an swa_status code and never throw. All validation happens before
+ *    any work is enqueued, so a non-OK return has enqueued nothing; the reason is in
+ *    swa_last_error(). A failure detected inside a kernel (a pipeline wait that ran
+ *    past its time limit, a negative decode position) is recorded in a per-device
+ *    status word and reported by swa_device_status().
+ *  - `out` must not alias q, k, v (or the rings); this is documented, not checked.
+ *  - Results are deterministic: the same inputs and sizes give bitwise-identical
+ *    outputs on every run.
+ */
+#ifndef SWA_H
+#define SWA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { SWA_F32 = 0, SWA_BF16 = 1 } swa_dtype;
+
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_INVALID_ARG = 1, /* bad size, window, dtype or null pointer */
+    SWA_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement (e.g. bf16 D=96) */
+    SWA_ERR_MISALIGNED = 3,  /* a pointer is not aligned as the kernel needs */
+    SWA_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed */
+    SWA_ERR_TIMEOUT = 5      /* a kernel wait ran past its limit (reported by swa_device_status) */
+} swa_status;
+
+/*
+ * swa_forward: prefill. out[B,H,T,D] = sliding-window causal attention of q, k, v.
+ *
+ *   q, k, v, out : [B, H, T, D] contiguous, all of `dtype`. Element (b,h,t,d) is at
+ *                  ((b*H + h)*T + t)*D + d. (A (B,T,H,D) caller transposes first; a
+ *                  3-D (B,T,D) input is H = 1.)
+ *   W            : window, W >= 1. W >= T is ordinary causal attention; W = 1 returns v.
+ *   dtype        : SWA_BF16 - bf16 in and out, fp32 accumulation, tensor cores
+ *                  (tcgen05), D must be 64 or 128, pointers 16-byte aligned;
+ *                  SWA_F32  - fp32 in and out, fp32 arithmetic on the CUDA cores
+ *                  (no TF32), any 1 <= D <= 4096, pointers 4-byte aligned.
+ *   scale        : 1/sqrt(D), fixed.
+ * Errors: W < 1, a negative size, D < 1, a null pointer (unless B*H*T == 0) or a bad
+ * dtype -> SWA_ERR_INVALID_ARG; B*H*T == 0 -> SWA_OK with nothing enqueued; an
+ * unsupported D or sizes beyond 2^31-1 rows -> SWA_ERR_UNSUPPORTED; misaligned
+ * pointers -> SWA_ERR_MISALIGNED; a failed launch -> SWA_ERR_CUDA.
+ */
+int swa_forward(const void* q, const void* k, const void* v, void* out,
+                int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                int dtype, void* stream);
+
+/*
+ * swa_decode: one new query per stream against a W-slot rolling KV buffer.
+ *
+ * "25. Sliding-Window Causal Attention for Streaming Inference" (Problem) pairs the
+ * window with a bounded KV cache that drops anything older than the window. Here the
+ * cache of stream b holds position p in slot p mod W. pos[b] is the 0-based absolute
+ * position of stream b's new query; the caller has already written that position's
+ * k and v into slot pos[b] mod W. The query attends to positions
+ * max(0, pos[b]-W+1) .. pos[b], which always occupy slots 0 .. min(pos[b]+1, W)-1.
+ * Slots outside that range are never read.
+ *
+ *   q, out       : [B, H, D] bf16.
+ *   kring, vring : [B, H, W, D] bf16; slot s of (b,h) starts at ((b*H + h)*W + s)*D.
+ *   pos          : [B] int64, on the device, each >= 0.
+ *   D            : 64 or 128. All pointers 16-byte aligned (pos 8-byte aligned).
+ * The work is split along the ring into chunks whose partial softmax states are merged
+ * in a fixed order (deterministic). The partial states live in a workspace that the
+ * library allocates with cudaMalloc on the first call for each (device, stream) and
+ * keeps, growing it when a larger call needs more: make that first call before any
+ * stream capture. Calls on one stream share its workspace; calls on different
+ * streams do not.
+ * Errors: as swa_forward; a negative pos[b] is found on the device: that stream's
+ * output is written as zeros and swa_device_status() reports SWA_ERR_INVALID_ARG.
+ */
+int swa_decode(const void* q, const void* kring, const void* vring, const int64_t* pos,
+               void* out, int64_t B, int64_t H, int64_t D, int64_t W, void* stream);
+
+/*
+ * swa_device_status: synchronize `stream`, then read and clear the current device's
+ * status word. Returns SWA_OK, or the first error a kernel recorded since the last
+ * call (SWA_ERR_TIMEOUT, SWA_ERR_INVALID_ARG), or SWA_ERR_CUDA if the synchronize or
+ * the read fails (the CUDA error string is then in swa_last_error()).
+ */
+int swa_device_status(void* stream);
+
+/* swa_last_error: message for the calling thread's last non-OK return ("" if none).
+ * The pointer stays valid until the thread's next call into the library. */
+const char* swa_last_error(void);
+
+/* ---- Host-side work planning (no GPU needed; the kernels use the same code) ---- */
+
+/*
+ * swa_prefill_tile_class: how the tensor-core prefill treats the key tile kt for
+ * the query tile qt, with query tiles of bm rows and key tiles of bn keys:
+ *   0 - not visited (no query row of the tile has a key of the tile in its band),
+ *   1 - edge tile (visited and masked element by element),
+ *   2 - full tile (every (i, j) pair of the tile is in the band and j < T; no mask).
+ * Visited tiles are kt_first .. kt_last with kt_first = max(0, qt*bm - W + 1) / bn and
+ * kt_last = min(T - 1, qt*bm + bm - 1) / bn: only the tiles that meet the band, as
+ * "NNX Sliding-Window Attention" (A local mask is not a sparse implementation) asks
+ * of an implementation that does O(T * min(W, T) * D) work. The kernels use bm = bn = 128.
+ * Returns -1 for invalid arguments (T < 1, W < 1, bm or bn < 1, qt or kt < 0,
+ * qt*bm >= T).
+ */
+int swa_prefill_tile_class(int64_t T, int64_t W, int64_t bm, int64_t bn, int64_t qt, int64_t kt);
+
+/*
+ * swa_decode_valid_slots: number n of ring slots that hold in-window positions for a
+ * stream at position pos: n = min(pos + 1, W); the valid slots are 0 .. n-1.
+ * Returns -1 if pos < 0 or W < 1.
+ */
+int64_t swa_decode_valid_slots(int64_t pos, int64_t W);
+
+/*
+ * swa_decode_split_plan: how swa_decode splits each stream's ring for B*H streams:
+ * writes the number of chunks per (b,h) and the chunk length in slots. Returns
+ * SWA_OK or SWA_ERR_INVALID_ARG.
+ */
+int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W,
+                          int32_t* splits, int32_t* chunk);
+
+/* ---- Diagnostics ---- */
+
+/*
+ * swa_set_wait_limit_ns: time limit of every bounded wait inside the kernels, in
+ * nanoseconds (default 2e9, or the SWA_WAIT_LIMIT_NS environment variable). A wait
+ * that runs past it makes the kernel record SWA_ERR_TIMEOUT, let its in-flight copies
+ * and tensor-core operations finish, free its tensor memory and return. 0 restores
+ * the default. Returns the previous limit.
+ */
+uint64_t swa_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * swa_timeout_probe: launch one CTA that waits on an mbarrier nothing ever arrives on,
+ * under the current wait limit, so that the timeout path can be tested without a
+ * fault or a hang. Afterwards swa_device_status() returns SWA_ERR_TIMEOUT.
+ */
+int swa_timeout_probe(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H */

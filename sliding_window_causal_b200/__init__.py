@@ -1,1 +1,157 @@
-"""Sliding-window causal attention for B200 (sm_100a)."""
+"""Sliding-window causal attention for B200 (sm_100a).
+
+Query i attends to keys j with 0 <= i - j < W. The CUDA library behind include/swa.h
+does all the work; these functions check torch tensors, pass their device pointers
+and the current CUDA stream to the C ABI, and raise SwaError on a non-OK status.
+PyTorch only supplies device memory and streams.
+
+    forward(q, k, v, window)            prefill, q/k/v [B,H,T,D] bf16 (D 64|128) or fp32
+    decode(q, kring, vring, pos, window)  one query per stream over a W-slot ring
+    forward_host(...)                   prefill from pinned host tensors (copies included)
+"""
+import ctypes
+
+from . import _native
+from ._native import SWA_BF16, SWA_F32, SwaError, check
+
+__all__ = ["forward", "decode", "forward_host", "device_status", "tile_class", "valid_slots",
+           "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(device):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return SWA_BF16
+    if t.dtype == torch.float32:
+        return SWA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (use forward_host for host tensors)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    dev = ts[0].device
+    if any(t.device != dev for t in ts):
+        raise ValueError("tensors must be on one device")
+    return dev
+
+
+def forward(q, k, v, window, out=None):
+    """Sliding-window causal attention prefill. q, k, v: [B,H,T,D] contiguous CUDA
+    tensors of one dtype (bf16 with D in {64, 128}, or fp32 with any D <= 4096).
+    A 3-D [B,T,D] input is treated as one head. Returns out (same shape and dtype)."""
+    torch = _torch()
+    squeeze = q.dim() == 3
+    if squeeze:
+        q, k, v = q.unsqueeze(1), k.unsqueeze(1), v.unsqueeze(1)
+        if out is not None:
+            out = out.unsqueeze(1)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B,H,T,D] shape")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    dev = _need_cuda(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need_cuda(out)
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out must match q")
+    B, H, T, D = q.shape
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        B, H, T, D, int(window), _dtype_code(q), _stream_ptr(dev)))
+    return out.squeeze(1) if squeeze else out
+
+
+def decode(q, kring, vring, pos, window, out=None):
+    """One new query per stream over a W-slot rolling KV buffer (slot = position mod W).
+    q: [B,H,D] bf16; kring, vring: [B,H,W,D] bf16; pos: [B] int64 on the device (the
+    0-based position of each stream's query, whose k/v are already in slot pos mod W)."""
+    torch = _torch()
+    if q.dim() != 3 or kring.dim() != 4:
+        raise ValueError("q must be [B,H,D] and the rings [B,H,W,D]")
+    B, H, D = q.shape
+    if kring.shape != (B, H, window, D) or vring.shape != kring.shape:
+        raise ValueError("rings must be [B,H,W,D] with W = window")
+    if pos.shape != (B,) or pos.dtype != torch.int64:
+        raise ValueError("pos must be int64 [B]")
+    if q.dtype != torch.bfloat16 or kring.dtype != torch.bfloat16 or vring.dtype != torch.bfloat16:
+        raise TypeError("decode takes bf16 q and rings")
+    dev = _need_cuda(q, kring, vring, pos)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need_cuda(out)
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_decode(q.data_ptr(), kring.data_ptr(), vring.data_ptr(),
+                                       pos.data_ptr(), out.data_ptr(), B, H, D, int(window),
+                                       _stream_ptr(dev)))
+    return out
+
+
+def forward_host(q, k, v, window, out=None, device=None, staging=None):
+    """Prefill from host tensors: copy q, k, v to the device on the current stream,
+    run forward, copy the result back into `out` (pinned host memory recommended).
+    `staging` may hold preallocated device tensors (q, k, v, out) to reuse."""
+    torch = _torch()
+    device = torch.device(device or "cuda")
+    if staging is None:
+        staging = tuple(torch.empty(q.shape, dtype=q.dtype, device=device) for _ in range(4))
+    dq, dk, dv, dout = staging
+    dq.copy_(q, non_blocking=True)
+    dk.copy_(k, non_blocking=True)
+    dv.copy_(v, non_blocking=True)
+    forward(dq, dk, dv, window, out=dout)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    out.copy_(dout, non_blocking=True)
+    return out
+
+
+def device_status(stream=None):
+    """Synchronize the stream and return/clear the device status word (raises on error)."""
+    torch = _torch()
+    s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    return check(_native.lib().swa_device_status(s))
+
+
+def tile_class(T, W, bm, bn, qt, kt):
+    """0 not visited, 1 edge (masked), 2 full; -1 invalid. Host only, no GPU needed."""
+    return _native.lib().swa_prefill_tile_class(T, W, bm, bn, qt, kt)
+
+
+def valid_slots(pos, W):
+    """Number of valid ring slots (slots 0..n-1) for a stream at position pos."""
+    return _native.lib().swa_decode_valid_slots(pos, W)
+
+
+def split_plan(B, H, D, W):
+    """(splits, chunk) that swa_decode uses for these sizes."""
+    s, c = ctypes.c_int32(), ctypes.c_int32()
+    check(_native.lib().swa_decode_split_plan(B, H, D, W, ctypes.byref(s), ctypes.byref(c)))
+    return s.value, c.value
+
+
+def set_wait_limit_ns(ns):
+    """Set the kernels' bounded-wait limit (0 = default); returns the previous limit."""
+    return _native.lib().swa_set_wait_limit_ns(int(ns))
+
+
+def timeout_probe():
+    """Launch the kernel whose wait never completes, to exercise the timeout path."""
+    torch = _torch()
+    check(_native.lib().swa_timeout_probe(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))

@@ -1,0 +1,114 @@
+"""C-ABI library on the CPU: it loads, exports every symbol include/swa.h declares, and
+its host-side work planning (tile classification, ring slots, decode splits) is
+bit-exact against brute-force enumeration. No GPU compute is called here."""
+import itertools
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sliding_window_causal_b200 as swa
+from sliding_window_causal_b200 import _native, build
+from oracle import brute
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    build.build()
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "swa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(swa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = header_symbols()
+    assert set(names) == set(_native.EXPORTS), "binding list and header disagree"
+    h = _native.lib()
+    for n in names:
+        assert hasattr(h, n), f"{n} not exported"
+
+
+def test_exports_are_c_linkage():
+    out = os.popen(f"nm -D --defined-only {_native.LIB_PATH}").read()
+    for n in header_symbols():
+        assert re.search(rf"\sT {n}$", out, flags=re.M), f"{n} missing or mangled"
+
+
+def _brute_tile_class(T, W, bm, bn, qt, kt):
+    """Enumerate every (i, j) pair of the tile: band membership for real rows decides
+    'visited', and 'full' means every pair of the tile (padding rows included) is in
+    the band with j < T."""
+    mask = brute.band_mask(max(T, (qt + 1) * bm, (kt + 1) * bn), W)
+    rows = range(qt * bm, qt * bm + bm)
+    cols = range(kt * bn, kt * bn + bn)
+    visited = any(mask[i, j] for i in rows if i < T for j in cols if j < T)
+    if not visited:
+        return 0
+    full = all(mask[i, j] and j < T for i in rows for j in cols)
+    return 2 if full else 1
+
+
+@pytest.mark.parametrize("bm,bn", [(4, 4), (4, 8), (8, 4), (3, 5)])
+def test_tile_class_matches_brute_force(bm, bn):
+    for T in (1, 2, 5, 8, 13, 24):
+        for W in (1, 2, 3, 4, 7, 8, 9, 16, 30):
+            for qt in range((T + bm - 1) // bm):
+                for kt in range((T + bn - 1) // bn + 1):
+                    got = swa.tile_class(T, W, bm, bn, qt, kt)
+                    assert got == _brute_tile_class(T, W, bm, bn, qt, kt), (T, W, bm, bn, qt, kt)
+
+
+def test_tile_class_kernel_tiles():
+    """The kernels' 128 x 128 tiles: every in-band pair lies in a visited tile, and
+    tiles flagged full hold only in-band pairs (checked by counting)."""
+    bm = bn = 128
+    for T, W in [(130, 1), (300, 129), (1000, 128), (1000, 127), (520, 4096), (777, 300)]:
+        mask = brute.band_mask(T, W) if T <= 1000 else None
+        nq = (T + bm - 1) // bm
+        covered = np.zeros((T, T), dtype=bool)
+        for qt in range(nq):
+            for kt in range(nq):
+                c = swa.tile_class(T, W, bm, bn, qt, kt)
+                r = slice(qt * bm, min(T, qt * bm + bm))
+                s = slice(kt * bn, min(T, kt * bn + bn))
+                if c:
+                    covered[r, s] = True
+                    assert mask[r, s].any(), "visited tile without an in-band pair"
+                if c == 2:
+                    assert mask[r, s].all() and kt * bn + bn <= T
+        assert not (mask & ~covered).any(), "in-band pair outside the visited tiles"
+
+
+def test_tile_class_rejects_bad_args():
+    assert swa.tile_class(0, 3, 128, 128, 0, 0) == -1
+    assert swa.tile_class(100, 0, 128, 128, 0, 0) == -1
+    assert swa.tile_class(100, 3, 128, 128, 1, 0) == -1
+
+
+def test_valid_slots_match_ring_enumeration():
+    for W in (1, 2, 3, 7, 64):
+        for pos in list(range(0, 3 * W + 2)) + [W - 2, W - 1, W, 10**6 + 3]:
+            if pos < 0:
+                continue
+            n = swa.valid_slots(pos, W)
+            held = brute.ring_positions(pos, W)
+            slots = sorted(s for _, s in held)
+            assert slots == list(range(n)), (pos, W)
+            assert n == min(pos + 1, W)
+    assert swa.valid_slots(-1, 4) == -1
+    assert swa.valid_slots(3, 0) == -1
+
+
+def test_split_plan_covers_window():
+    for (B, H, D, W) in itertools.product((1, 3, 64), (1, 32), (64, 128), (1, 31, 4096, 5000)):
+        S, chunk = swa.split_plan(B, H, D, W)
+        assert S >= 1 and chunk >= 1
+        assert (S - 1) * chunk < W <= S * chunk
+    with pytest.raises(swa.SwaError):
+        swa.split_plan(1, 1, 96, 10)

@@ -1,0 +1,202 @@
+"""GPU prefill (swa_forward through the C ABI) against the float64 oracle."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_causal_b200 as swa
+from sliding_window_causal_b200 import _native, inputs
+from golden import read_moving_average
+from gpu_util import TOL, f64, max_err, oracle_rows, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run(q, k, v, W):
+    out = swa.forward(q.to(DEV), k.to(DEV), v.to(DEV), W)
+    swa.device_status()
+    return out
+
+
+def full_parity(B, H, T, D, W, dtype, seed):
+    q, k, v = inputs.prefill_inputs(B, H, T, D, dtype, seed)
+    out = run(q, k, v, W)
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    err = max_err(out, ref)
+    assert err <= TOL[dtype], f"max err {err} (B{B} H{H} T{T} D{D} W{W} {dtype})"
+    return err
+
+
+@pytest.mark.parametrize("wl", inputs.TINY, ids=lambda w: w.name)
+def test_tiny_fp32_workload(wl):
+    full_parity(wl.B, wl.H, wl.T, wl.D, wl.W, wl.dtype, wl.seed)
+
+
+def test_small_bf16_workload():
+    wl = inputs.SMALL
+    full_parity(wl.B, wl.H, wl.T, wl.D, wl.W, wl.dtype, wl.seed)
+
+
+BF16_SHAPES = [
+    # B, H, T, D, W: ragged T, W below/at/above a tile, W >= T, single rows
+    (1, 2, 300, 64, 1), (1, 2, 300, 64, 77), (2, 2, 1000, 128, 128), (1, 3, 1000, 128, 127),
+    (1, 2, 1000, 128, 129), (1, 2, 777, 128, 300), (1, 1, 1000, 128, 1000),
+    (1, 1, 1000, 128, 5000), (1, 2, 129, 64, 2), (1, 1, 1, 128, 1), (1, 1, 5, 64, 3),
+    (2, 3, 400, 64, 256), (1, 1, 2000, 128, 640), (1, 2, 1280, 64, 1),
+]
+
+
+@pytest.mark.parametrize("B,H,T,D,W", BF16_SHAPES)
+def test_bf16_parity(B, H, T, D, W):
+    full_parity(B, H, T, D, W, torch.bfloat16, 7 + T + W)
+
+
+FP32_SHAPES = [(1, 2, 6, 4, 3), (2, 3, 100, 1, 7), (1, 2, 257, 33, 40), (1, 1, 300, 128, 300),
+               (1, 2, 70, 200, 1000), (1, 1, 40, 1100, 9)]
+
+
+@pytest.mark.parametrize("B,H,T,D,W", FP32_SHAPES)
+def test_fp32_parity(B, H, T, D, W):
+    full_parity(B, H, T, D, W, torch.float32, 3 + T + W)
+
+
+def test_moving_average_example_exact():
+    """The printed moving-average example (two heads of width 1, window 3, zero q and
+    k) comes out exactly, and changing input row 0 leaves rows 3+ unchanged."""
+    g = read_moving_average()
+    x = torch.tensor(g["x"], dtype=torch.float32)
+    T, Hn = x.shape
+    v = x.t().reshape(1, Hn, T, 1).contiguous()
+    z = torch.zeros_like(v)
+    out = run(z, z, v, g["W"])[0, :, :, 0].t().cpu()
+    assert torch.equal(out, torch.tensor(g["y"], dtype=torch.float32))
+    row, vals = g["changed_row"]
+    x2 = x.clone()
+    x2[row] = torch.tensor(vals)
+    v2 = x2.t().reshape(1, Hn, T, 1).contiguous()
+    out2 = run(z, z, v2, g["W"])[0, :, :, 0].t().cpu()
+    u = g["unchanged_from"]
+    assert torch.equal(out2[u:], out[u:])
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 5)])
+def test_window_one_returns_v_bitwise(dtype, D):
+    q, k, v = inputs.prefill_inputs(2, 2, 333, D, dtype, 11)
+    out = run(q, k, v, 1).cpu()
+    assert torch.equal(out, v)
+
+
+def test_window_at_least_T_is_causal():
+    """W >= T equals ordinary causal attention (the oracle with W = T), and every
+    W >= T gives the same bits."""
+    q, k, v = inputs.prefill_inputs(1, 2, 500, 128, torch.bfloat16, 13)
+    ref = oracle.forward(f64(q), f64(k), f64(v), 500)
+    a = run(q, k, v, 500)
+    b = run(q, k, v, 10**9)
+    assert max_err(a, ref) <= TOL[torch.bfloat16]
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_out_of_band_corruption_bitwise(D):
+    """Corrupt-and-compare: changing k and v (finite values) at positions j <= i0 - W
+    leaves every row i >= i0 bitwise unchanged."""
+    T, W, i0 = 1000, 100, 700
+    q, k, v = inputs.prefill_inputs(1, 2, T, D, torch.bfloat16, 17)
+    base = run(q, k, v, W).cpu()
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, : i0 - W + 1] = 100.0
+    v2[:, :, : i0 - W + 1] = -200.0
+    out = run(q, k2, v2, W).cpu()
+    assert torch.equal(out[:, :, i0:], base[:, :, i0:])
+    assert not torch.equal(out[:, :, :i0], base[:, :, :i0])
+
+
+def test_deterministic():
+    q, k, v = inputs.prefill_inputs(1, 4, 1500, 128, torch.bfloat16, 19)
+    a = run(q, k, v, 600)
+    b = run(q, k, v, 600)
+    assert torch.equal(a, b)
+
+
+def test_three_dim_input_is_one_head():
+    q = torch.randn(1, 5, 3, generator=torch.Generator().manual_seed(5))
+    out = swa.forward(q.to(DEV), q.to(DEV), q.to(DEV), 2)
+    swa.device_status()
+    assert out.shape == (1, 5, 3)
+    ref = oracle.forward(f64(q)[:, None], f64(q)[:, None], f64(q)[:, None], 2)[:, 0]
+    assert max_err(out, ref) <= TOL[torch.float32]
+
+
+def test_empty_inputs_are_noops():
+    for shape in [(0, 2, 16, 64), (1, 0, 16, 64), (1, 2, 0, 64)]:
+        q = torch.zeros(shape, dtype=torch.bfloat16, device=DEV)
+        out = swa.forward(q, q, q, 4)
+        assert out.shape == shape
+    swa.device_status()
+
+
+def test_argument_errors():
+    h = _native.lib()
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16, device=DEV)
+    p = q.data_ptr()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert h.swa_forward(p, p, p, p, 1, 1, 8, 64, 0, 1, s) == 1  # W < 1
+    assert b"W=0" in h.swa_last_error()
+    assert h.swa_forward(p, p, p, p, 1, 1, 8, 64, 3, 7, s) == 1  # dtype
+    assert h.swa_forward(p, p, p, p, -1, 1, 8, 64, 3, 1, s) == 1  # negative size
+    assert h.swa_forward(None, p, p, p, 1, 1, 8, 64, 3, 1, s) == 1  # null
+    assert h.swa_forward(p, p, p, p, 1, 1, 8, 96, 3, 1, s) == 2  # bf16 D=96
+    assert h.swa_forward(p + 2, p, p, p, 1, 1, 4, 64, 3, 1, s) == 3  # misaligned
+    with pytest.raises(swa.SwaError):
+        swa.forward(q, q, q, 0)
+    swa.device_status()
+
+
+def test_timeout_path_reports_and_recovers():
+    """A wait that nothing completes runs out and is reported, and the context
+    stays usable for the next calls."""
+    prev = swa.set_wait_limit_ns(20_000_000)
+    try:
+        swa.timeout_probe()
+        with pytest.raises(swa.SwaError) as ei:
+            swa.device_status()
+        assert ei.value.code == 5
+    finally:
+        swa.set_wait_limit_ns(0)
+    full_parity(1, 2, 300, 128, 100, torch.bfloat16, 23)
+    swa.device_status()
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+def sampled_parity(wl, heads, n_random=96):
+    q, k, v = inputs.for_workload(wl)
+    out = swa.forward(q.to(DEV), k.to(DEV), v.to(DEV), wl.W)
+    swa.device_status()
+    rows = sample_rows(wl.T, wl.W, n_random=n_random, seed=wl.seed)
+    refs = oracle_rows(q, k, v, wl.W, heads, rows)
+    worst = 0.0
+    for (b, h), ref in refs.items():
+        got = out[b, h, torch.from_numpy(rows).to(DEV)]
+        worst = max(worst, max_err(got, ref))
+    assert worst <= TOL[wl.dtype], f"{wl.name}: max err {worst}"
+    # properties at any size, over every output: finite, and each output a convex
+    # combination of v rows, so no larger in magnitude than the largest |v|
+    assert bool(torch.isfinite(out).all())
+    vmax = v.abs().max().item()
+    assert out.abs().max().item() <= vmax * (1 + 2 ** -8)
+    return worst
+
+
+def test_mistral_shaped_sampled():
+    wl = inputs.MISTRAL
+    sampled_parity(wl, [(0, 0), (0, 13), (0, 31)])
+
+
+@pytest.mark.parametrize("wl", inputs.SWEEP, ids=lambda w: w.name)
+def test_window_sweep_sampled(wl):
+    sampled_parity(wl, [(0, 0), (1, 15)], n_random=48)
