@@ -196,6 +196,17 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def prefill_workload(name):
+    if name == "mistral":
+        return inputs.MISTRAL
+    if name == "small":
+        return inputs.SMALL
+    for w in inputs.SWEEP:
+        if name == f"sweep-w{w.W}":
+            return w
+    raise SystemExit(f"unknown workload {name}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -204,6 +215,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default="mistral",
+                    help="prefill workload of the main line: mistral (default), small, "
+                         "sweep-w{1,256,1024,4096,8192}")
+    ap.add_argument("--decode-streams", type=int, default=None,
+                    help="override the decode workload's stream count (smaller profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -223,7 +240,7 @@ def main():
     peak_tf, peak_gbs, peak_kind = load_peaks()
 
     # ------------------------------------------------------------ prefill
-    wl = inputs.MISTRAL
+    wl = prefill_workload(args.workload)
     qh, kh, vh = inputs.for_workload(wl)
     q, k, v = (t.to(device) for t in (qh, kh, vh))
     out = torch.empty_like(q)
@@ -242,20 +259,22 @@ def main():
     achieved = F / (ms_step * 1e-3) / 1e12
 
     # ------------------------------------------------------------ e2e (host buffers)
-    pin = lambda t: t.pin_memory()
-    qp, kp, vp = pin(qh), pin(kh), pin(vh)
-    outp = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+    e2e = None
     staging = (q, k, v, out)
-    e2e_fn = lambda: swa.forward_host(qp, kp, vp, wl.W, out=outp, device=device, staging=staging)
-    for _ in range(3):
-        e2e_fn()
-    e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms = timed(e2e_fn, e2e_steps, stream, pg, device) / e2e_steps
-    swa.device_status()
-    e2e_value = world * F / (e2e_ms * 1e-3) / 1e12
-    h2d = 3 * qh.numel() * qh.element_size()
-    d2h = outp.numel() * outp.element_size()
-    del qp, kp, vp, outp
+    if not args.no_e2e:
+        pin = lambda t: t.pin_memory()
+        qp, kp, vp = pin(qh), pin(kh), pin(vh)
+        outp = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+        e2e_fn = lambda: swa.forward_host(qp, kp, vp, wl.W, out=outp, device=device, staging=staging)
+        for _ in range(3):
+            e2e_fn()
+        e2e_steps = max(3, min(args.steps, 20))
+        e2e_ms = timed(e2e_fn, e2e_steps, stream, pg, device) / e2e_steps
+        swa.device_status()
+        e2e = {"value": world * F / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
+               "d2h_bytes_per_step": outp.numel() * outp.element_size(), "steps": e2e_steps}
+        del qp, kp, vp, outp
 
     # ------------------------------------------------------------ decode
     decode_line = None
@@ -263,6 +282,10 @@ def main():
         del q, k, v, out, staging
         torch.cuda.empty_cache()
         dw = inputs.DECODE
+        if args.decode_streams:
+            import dataclasses
+            dw = dataclasses.replace(dw, B=args.decode_streams,
+                                     name=dw.name.replace("B64", f"B{args.decode_streams}"))
         dq, dkr, dvr, dpos = inputs.for_workload(dw)
         nbytes = decode_bytes(dw.B, dw.H, dw.D, dw.W, dpos)
         dq, dkr, dvr, dpos = (t.to(device) for t in (dq, dkr, dvr, dpos))
@@ -280,7 +303,7 @@ def main():
             "metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": dms,
             "config": {"workload": dw.name, "B": dw.B, "H": dw.H, "D": dw.D, "W": dw.W,
                        "pos": "uniform [0, 100000)", "seed": dw.seed, "splits": S, "chunk": chunk,
-                       "l2": "inputs larger than L2 (4.3 GB of rings)"},
+                       "l2": f"inputs larger than L2 ({2 * dkr.numel() * 2 / 1e9:.2f} GB of rings)"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s",
                          "frac": gbs / peak_gbs, "peak_kind": peak_kind, "traffic": None,
                          "algorithmic_bytes": nbytes},
@@ -300,12 +323,12 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D, "W": wl.W,
                    "seed": wl.seed, "band_flops": F,
-                   "l2": "inputs larger than L2 (q, k, v 384 MB), no flush"},
+                   "l2": f"inputs larger than L2 (q, k, v {3 * qh.numel() * 2 / 2**20:.0f} MiB), no flush"
+                   if 3 * qh.numel() * 2 > L2_BYTES else "inputs smaller than L2: L2-resident"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": None, "frac_of_spec_2250": achieved / 2250.0},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,

@@ -37,6 +37,11 @@ namespace swa {
 constexpr int kTileM = 128;  // query rows per tile
 constexpr int kTileN = 128;  // keys per tile
 constexpr float kRescaleThreshold = 8.0f;  // lazy O rescale: max may grow by 2^8 first
+// Query tiles whose rows see few keys (the first tile of every head, or any tile when
+// W <= kPreciseWindow) carry P as a bf16 pair hi + lo (two P.V MMAs). There a couple of
+// weights decide each output, |out| can reach 2 and more, and the 2^-9 relative rounding
+// of a single bf16 P would use up most of the error budget left by the output rounding.
+constexpr int kPreciseWindow = 32;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr int kStatusTimeout = 5;  // SWA_ERR_TIMEOUT
 
@@ -98,6 +103,7 @@ __global__ void __launch_bounds__(192, 1)
     kv_tile_range(T, W, kTileM, kTileN, qt, &ktf64, &ktl64);
     const int kt_first = (int)ktf64;
     const int n_tiles = (int)(ktl64 - ktf64 + 1);
+    const bool precise = (qt == 0) || (W <= kPreciseWindow);
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_full, 1);
@@ -207,6 +213,13 @@ __global__ void __launch_bounds__(192, 1)
                                     umma::smem_desc(v_addr + kk * 2048, C::kBoxBytes, 1024), idesc_o,
                                     (jp > 0 || kk > 0) ? 1u : 0u);
                     }
+                    if (precise) {  // low halves of P, stored 64 columns further on
+#pragma unroll
+                        for (int kk = 0; kk < kTileN / 16; ++kk)
+                            ptx::mma_ts(tmem + C::kColO, tmem + C::colS(bp) + 64 + kk * 8,
+                                        umma::smem_desc(v_addr + kk * 2048, C::kBoxBytes, 1024),
+                                        idesc_o, 1u);
+                    }
                     ptx::tc_commit(v_empty + st);
                     ptx::tc_commit(o_done);
                     if (jp == n_tiles - 1) ptx::tc_commit(o_final);
@@ -289,22 +302,35 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            uint32_t p[2][32];
+            // P in chunks of 16 packed pairs (32 keys), each stored as soon as it is
+            // ready; the row sum counts exactly the bf16 weights the MMA multiplies by.
             float ls0 = 0.f, ls1 = 0.f;
+            __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float e0 = ptx::ex2(fmaf(sv[2 * c], scale_log2, -m_use));
-                const float e1 = ptx::ex2(fmaf(sv[2 * c + 1], scale_log2, -m_use));
-                const uint32_t pk = ptx::pack_bf16x2(e0, e1);
-                p[c >> 5][c & 31] = pk;
-                // the row sum counts exactly the bf16 weights the MMA multiplies by
-                ls0 += ptx::bf16lo_f32(pk);
-                ls1 += ptx::bf16hi_f32(pk);
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t ph[16], pl[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int cp = q4 * 16 + c;
+                    const float e0 = ptx::ex2(fmaf(sv[2 * cp], scale_log2, -m_use));
+                    const float e1 = ptx::ex2(fmaf(sv[2 * cp + 1], scale_log2, -m_use));
+                    const uint32_t hi = ptx::pack_bf16x2(e0, e1);
+                    const float h0 = ptx::bf16lo_f32(hi), h1 = ptx::bf16hi_f32(hi);
+                    ph[c] = hi;
+                    if (precise) {
+                        const uint32_t lo = ptx::pack_bf16x2(e0 - h0, e1 - h1);
+                        pl[c] = lo;
+                        ls0 += h0 + ptx::bf16lo_f32(lo);
+                        ls1 += h1 + ptx::bf16hi_f32(lo);
+                    } else {
+                        ls0 += h0;
+                        ls1 += h1;
+                    }
+                }
+                ptx::tmem_st16(tl + C::colS(b) + q4 * 16, ph);
+                if (precise) ptx::tmem_st16(tl + C::colS(b) + 64 + q4 * 16, pl);
             }
             l += ls0 + ls1;
-            __syncwarp();
-            ptx::tmem_st32(tl + C::colS(b), p[0]);
-            ptx::tmem_st32(tl + C::colS(b) + 32, p[1]);
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full + b);

@@ -142,34 +142,50 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t BH, int64_t T, int64_t D) 
 }
 
 // ------------------------------------------------------------------ decode workspace
+// Per (device, stream): the split partial states (m, l, acc[D]) and, in a separate
+// allocation, one ticket counter per stream. Every counter is zero between calls: the
+// allocation is zeroed and the last CTA of each stream resets its counter.
 struct Workspace {
-    void* ptr = nullptr;
-    size_t bytes = 0;
+    void* part = nullptr;
+    size_t part_bytes = 0;
+    int* counters = nullptr;
+    size_t n_counters = 0;
 };
 std::map<std::pair<int, void*>, Workspace> g_ws;
 
-int decode_workspace(void* stream, size_t need, void** out) {
+int decode_workspace(void* stream, size_t part_need, size_t counters_need, float** part,
+                     int** counters) {
     int dev;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace& w = g_ws[std::make_pair(dev, stream)];
-    if (w.bytes < need) {
-        cudaStream_t s = static_cast<cudaStream_t>(stream);
-        if (w.ptr) {
-            e = cudaStreamSynchronize(s);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-            cudaFree(w.ptr);
-            w.ptr = nullptr;
-            w.bytes = 0;
-        }
-        e = cudaMalloc(&w.ptr, need);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(decode workspace)");
-        e = cudaMemsetAsync(w.ptr, 0, need, s);  // ticket counters start at zero
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-        w.bytes = need;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (w.part_bytes < part_need || w.n_counters < counters_need) {
+        // the stream may still be using the old buffers
+        e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     }
-    *out = w.ptr;
+    if (w.part_bytes < part_need) {
+        if (w.part) cudaFree(w.part);
+        w.part = nullptr;
+        w.part_bytes = 0;
+        e = cudaMalloc(&w.part, part_need);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(decode partials)");
+        w.part_bytes = part_need;
+    }
+    if (w.n_counters < counters_need) {
+        if (w.counters) cudaFree(w.counters);
+        w.counters = nullptr;
+        w.n_counters = 0;
+        e = cudaMalloc(&w.counters, counters_need * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(decode counters)");
+        e = cudaMemsetAsync(w.counters, 0, counters_need * sizeof(int), s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+        w.n_counters = counters_need;
+    }
+    *part = static_cast<float*>(w.part);
+    *counters = w.counters;
     return SWA_OK;
 }
 
@@ -305,11 +321,8 @@ int swa_decode(const void* q, const void* kring, const void* vring, const int64_
     int* counters = nullptr;
     if (S > 1) {
         const size_t part_bytes = (size_t)(B * H) * S * (D + 2) * sizeof(float);
-        const size_t need = part_bytes + (size_t)(B * H) * sizeof(int);
-        void* ws;
-        if (int rc = decode_workspace(stream, need, &ws)) return rc;
-        part = static_cast<float*>(ws);
-        counters = reinterpret_cast<int*>(static_cast<char*>(ws) + part_bytes);
+        if (int rc = decode_workspace(stream, part_bytes, (size_t)(B * H), &part, &counters))
+            return rc;
     }
     const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     const dim3 grid((unsigned)(B * H), (unsigned)S);

@@ -125,3 +125,15 @@ def test_streaming_decode_workload_sampled():
                             f64(vr[b:b + 1, h:h + 1]), pos[b:b + 1].numpy(), wl.W)
         worst = max(worst, max_err(out[b:b + 1, h:h + 1], ref))
     assert worst <= TOL_BF16, f"max err {worst}"
+
+
+def test_workspace_reuse_across_sizes():
+    """Calls of different sizes on one stream share the library's workspace: a large
+    call followed by smaller ones (fewer streams, other split counts) stays exact."""
+    cases = [(24, 3, 128, 3000), (2, 1, 128, 200), (5, 2, 64, 700), (1, 2, 128, 4096),
+             (24, 3, 128, 3000)]
+    for i, (B, H, D, W) in enumerate(cases):
+        q, kr, vr, pos = inputs.decode_inputs(B, H, D, W, 5 * W, torch.bfloat16, 60 + i)
+        out = run(q, kr, vr, pos, W)
+        ref = oracle.decode(f64(q), f64(kr), f64(vr), pos.numpy(), W)
+        assert max_err(out, ref) <= TOL_BF16, (B, H, D, W)
