@@ -1,0 +1,485 @@
+// prefill_pp.cuh: persistent, ping-pong bf16 sliding-window causal attention prefill on
+// the sm_100a tensor cores.
+//
+// Work items are pairs of consecutive 128-row query tiles (A = 2p, B = 2p+1) of one (b,h).
+// Both tiles meet nearly the same 128-key tiles of the band, so every K and V tile is
+// loaded once for the pair. Only the key tiles that meet a tile's band are computed for
+// it, and only edge tiles are masked ("NNX Sliding-Window Attention", A local mask is not
+// a sparse implementation: only the allowed windows need computing).
+//
+// The grid holds at most one CTA per SM; CTA g takes items g, then 2G-1-g, then 2G+g, ...
+// of the list ordered heaviest first (a snake over the list), which balances the load
+// without any device-side queue.
+//
+// Roles (320 threads, one CTA per SM):
+//   warp 0, lane 0     TMA producer: Q_A, Q_B per item, then K_kt and V_kt through one
+//                      NSTAGE-deep ring of 128-row tiles.
+//   warp 1             allocates the 512 TMEM columns; lane 0 issues every tcgen05 MMA in
+//                      the order PV_A(kt-1), S_A(kt), PV_B(kt-1), S_B(kt), so that the tensor
+//                      core works on one tile's products while the other tile's softmax runs:
+//                        S_X = Q_X K^T   -> TMEM columns [128X, 128X+128)   (fp32)
+//                        O_X += P_X V    -> TMEM columns [256+128X, +D)     (fp32)
+//   warps 2..5 (A), 6..9 (B)    softmax of one query tile each, one row per thread (warp w
+//                      reads TMEM lanes 32*(w%4)..): running max and sum of the online
+//                      softmax ("Mistral Architecture > Implementation: Sliding Window
+//                      Attention", Step 2, stable softmax), -inf select on edge tiles, P
+//                      written over the S columns as bf16, lazy rescale of O, and finally
+//                      O/l rounded to bf16 and stored to global memory.
+// Because the MMAs of one thread complete in issue order, S_X(kt) completing implies that
+// PV_X(kt-1) is complete: the softmax may rescale O_X right after it sees S_X(kt).
+//
+// Every mbarrier wait is bounded by wait_limit_ns. A role that runs past it records
+// SWA_ERR_TIMEOUT, raises the CTA's abort flag (the other roles then stop waiting), and
+// the CTA lets its in-flight TMA loads and MMAs finish, frees its TMEM and returns.
+#pragma once
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "plan.h"
+#include "ptx.cuh"
+#include "umma.h"
+
+namespace swa {
+
+constexpr int kPPThreads = 320;
+constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow by 2^8 first
+// Query tiles whose rows see few keys (the first tile of every head, or any tile when
+// W <= kPPPreciseWindow) carry P as two bf16 parts hi + lo with a second P.V MMA: there a
+// couple of weights decide each output and |out| can exceed 2, so a single bf16 P would
+// use up the error budget left by the output's own bf16 rounding.
+constexpr int kPPPreciseWindow = 32;
+constexpr uint64_t kPPDrainLimitNs = 200000000ull;
+
+template <int D>
+struct PPCfg {
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 64 bf16
+    static constexpr int kTileBytes = 128 * D * 2;     // one 128-row tile of Q, K or V
+    static constexpr int kStages = D == 128 ? 5 : 12;  // unified K/V ring
+    static constexpr int kQOff = 0;                    // Q_A, Q_B
+    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+    // q_full[2], q_empty[2], ring_full[S], ring_empty[S], s_full[2], p_full[2],
+    // o_final[2], o_free[2], drain
+    static constexpr int kNumBars = 4 + 2 * kStages + 9;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+    static constexpr uint32_t kTmemCols = 512;
+    __device__ static constexpr uint32_t colS(int x) { return 128u * x; }
+    __device__ static constexpr uint32_t colO(int x) { return 256u + 128u * x; }
+};
+
+// The r-th item of CTA g among n items on G CTAs (snake order), or -1.
+__device__ __forceinline__ int pp_item(int r, int g, int G, int n) {
+    const int u = r * G + ((r & 1) ? (G - 1 - g) : g);
+    return u < n ? u : -1;
+}
+
+struct PPItem {
+    int bh, qt[2], f[2], l[2], k0, k1;
+    bool hasB;
+};
+
+__device__ __forceinline__ PPItem pp_decode(int u, int BH, int n_qt, int T, int W) {
+    PPItem it;
+    const int n_pairs = (n_qt + 1) >> 1;
+    const int p = n_pairs - 1 - u / BH;  // heaviest pairs first
+    it.bh = u % BH;
+    it.qt[0] = 2 * p;
+    it.qt[1] = 2 * p + 1;
+    it.hasB = it.qt[1] < n_qt;
+    int64_t f, l;
+    kv_tile_range(T, W, 128, 128, it.qt[0], &f, &l);
+    it.f[0] = (int)f;
+    it.l[0] = (int)l;
+    it.f[1] = it.l[1] = -1;
+    if (it.hasB) {
+        kv_tile_range(T, W, 128, 128, it.qt[1], &f, &l);
+        it.f[1] = (int)f;
+        it.l[1] = (int)l;
+    }
+    it.k0 = it.f[0];
+    it.k1 = it.hasB ? it.l[1] : it.l[0];
+    return it;
+}
+
+__device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W <= kPPPreciseWindow; }
+
+// Column of TMEM (relative to the S buffer) that holds P for keys 16kk..16kk+15: keys
+// 32c..32c+31 are packed into columns 32c..32c+15 (and, for precise tiles, the low parts
+// into 32c+16..32c+31), so that P only ever overwrites S values already read.
+__device__ __forceinline__ uint32_t pp_pcol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
+
+template <int D>
+__global__ void __launch_bounds__(kPPThreads, 1)
+    prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+                      int BH, int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
+                      int* status) {
+    using C = PPCfg<D>;
+    constexpr int NS = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* q_full = bars;            // [2]
+    uint64_t* q_empty = bars + 2;       // [2]
+    uint64_t* ring_full = bars + 4;     // [NS]
+    uint64_t* ring_empty = ring_full + NS;
+    uint64_t* s_full = ring_empty + NS;  // [2]
+    uint64_t* p_full = s_full + 2;       // [2]
+    uint64_t* o_final = p_full + 2;      // [2]
+    uint64_t* o_free = o_final + 2;      // [2]
+    uint64_t* drain = o_free + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = ((n_qt + 1) >> 1) * BH;
+    const int G = gridDim.x, g = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < 2; ++x) {
+            ptx::mbar_init(q_full + x, 1);
+            ptx::mbar_init(q_empty + x, 1);
+            ptx::mbar_init(s_full + x, 1);
+            ptx::mbar_init(p_full + x, 128);
+            ptx::mbar_init(o_final + x, 1);
+            ptx::mbar_init(o_free + x, 128);
+        }
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(ring_full + s, 1);
+            ptx::mbar_init(ring_empty + s, 1);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    uint32_t loads = 0;  // producer: K/V tiles issued so far
+    int nq[2] = {0, 0};  // producer: Q tiles issued per side
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ producer
+            bool ok = true;
+            for (int r = 0; ok; ++r) {
+                const int u = pp_item(r, g, G, n_items);
+                if (u < 0) break;
+                const PPItem it = pp_decode(u, BH, n_qt, T, W);
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (!ok || (x == 1 && !it.hasB)) break;
+                    if (nq[x] > 0) ok = ptx::mbar_wait(q_empty + x, (nq[x] - 1) & 1, wait_limit_ns, abort_flag);
+                    if (!ok) break;
+                    uint8_t* dst = smem + C::kQOff + x * C::kTileBytes;
+                    ptx::mbar_arrive_expect_tx(q_full + x, C::kTileBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        ptx::tma_load_3d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.bh);
+                    ++nq[x];
+                }
+                for (int kt = it.k0; kt <= it.k1 && ok; ++kt) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const uint32_t st = loads % NS;
+                        if (loads >= (uint32_t)NS)
+                            ok = ptx::mbar_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag);
+                        if (!ok) break;
+                        uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
+                        ptx::mbar_arrive_expect_tx(ring_full + st, C::kTileBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            ptx::tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, ring_full + st, c * 64,
+                                             kt * 128, it.bh);
+                        ++loads;
+                    }
+                }
+            }
+            if (!ok) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ MMA issuer
+            const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
+            const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
+            uint32_t L = 0;               // K/V tiles consumed so far (same count as the producer)
+            int ni[2] = {0, 0};           // items seen per side
+            uint32_t ns[2] = {0, 0};      // S tiles issued per side
+            bool ok = true;
+            for (int r = 0; ok; ++r) {
+                const int u = pp_item(r, g, G, n_items);
+                if (u < 0) break;
+                const PPItem it = pp_decode(u, BH, n_qt, T, W);
+                const int nx = it.hasB ? 2 : 1;
+                bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (x < nx && ok) ok = ptx::mbar_wait(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
+                }
+                if (!ok) break;
+                int pend[2] = {-1, -1};
+                bool first_pv[2] = {true, true};
+                const uint32_t Lbase = L;
+                for (int kt = it.k0; kt <= it.k1 + 1 && ok; ++kt) {
+                    const uint32_t j = (uint32_t)(kt - it.k0);
+                    const uint32_t Lk = Lbase + 2 * j, Lv = Lk - 1;
+                    if (kt <= it.k1) ok = ptx::mbar_wait(ring_full + Lk % NS, (Lk / NS) & 1, wait_limit_ns, abort_flag);
+                    if (ok && kt > it.k0) ok = ptx::mbar_wait(ring_full + Lv % NS, (Lv / NS) & 1, wait_limit_ns, abort_flag);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        if (x >= nx || !ok) break;
+                        if (pend[x] >= 0) {
+                            // PV_x(kt-1): needs P_x(kt-1), and O_x free if it starts the item
+                            ok = ptx::mbar_wait(p_full + x, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
+                            if (ok && first_pv[x] && ni[x] > 0)
+                                ok = ptx::mbar_wait(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
+                            if (!ok) break;
+                            ptx::tc_fence_after();
+                            const uint32_t v_addr = ptx::smem_u32(smem + C::kRingOff + (Lv % NS) * C::kTileBytes);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
+                                            umma::smem_desc(v_addr + kk * 2048, C::kBoxBytes, 1024), idesc_o,
+                                            (!first_pv[x] || kk > 0) ? 1u : 0u);
+                            if (prec[x]) {
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                umma::smem_desc(v_addr + kk * 2048, C::kBoxBytes, 1024), idesc_o, 1u);
+                            }
+                            first_pv[x] = false;
+                            if (pend[x] == it.l[x]) ptx::tc_commit(o_final + x);
+                            pend[x] = -1;
+                        }
+                        if (kt <= it.k1 && kt >= it.f[x] && kt <= it.l[x]) {
+                            // S_x(kt) = Q_x K(kt)^T
+                            const uint32_t q_addr = ptx::smem_u32(smem + C::kQOff + x * C::kTileBytes);
+                            const uint32_t k_addr = ptx::smem_u32(smem + C::kRingOff + (Lk % NS) * C::kTileBytes);
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+                                ptx::mma_ss(tmem + C::colS(x), umma::smem_desc(q_addr + off, 16, 1024),
+                                            umma::smem_desc(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                            }
+                            ptx::tc_commit(s_full + x);
+                            ++ns[x];
+                            if (kt == it.l[x]) ptx::tc_commit(q_empty + x);
+                            pend[x] = kt;
+                        }
+                    }
+                    if (!ok) break;
+                    if (kt <= it.k1) ptx::tc_commit(ring_empty + Lk % NS);  // K(kt) read by its S MMAs
+                    if (kt > it.k0) ptx::tc_commit(ring_empty + Lv % NS);   // V(kt-1) read by its PV MMAs
+                }
+                L = Lbase + 2u * (uint32_t)(it.k1 - it.k0 + 1);
+                ++ni[0];
+                if (it.hasB) ++ni[1];
+            }
+            if (!ok) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax A / B
+        const int x = (warp - 2) >> 2;   // 0: tile A, 1: tile B
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint32_t ns = 0;   // S tiles seen
+        int ni = 0;        // items seen
+        bool ok = true;
+        for (int rr = 0; ok; ++rr) {
+            const int u = pp_item(rr, g, G, n_items);
+            if (u < 0) break;
+            const PPItem it = pp_decode(u, BH, n_qt, T, W);
+            if (x == 1 && !it.hasB) continue;
+            const int qt = x ? it.qt[1] : it.qt[0];
+            const int fx = x ? it.f[1] : it.f[0];
+            const int lx = x ? it.l[1] : it.l[0];
+            const bool precise = pp_precise(qt, W);
+            const int i = qt * 128 + r;
+            int lo = i - W + 1;
+            if (lo < 0) lo = 0;
+            const int hi = i < T - 1 ? i : T - 1;
+            float m_ref = -INFINITY, l = 0.f;
+            for (int kt = fx; kt <= lx; ++kt) {
+                bool w = ptx::mbar_wait(s_full + x, ns & 1, wait_limit_ns, abort_flag);
+                ++ns;
+                if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const bool edge = tile_class(T, W, 128, 128, qt, kt) != 2;
+                const int cmin = lo - kt * 128, cmax = hi - kt * 128;
+                // pass 1: row max over the tile (masked on edge tiles)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t a[32], b2[32];
+                    ptx::tmem_ld32(tl + C::colS(x) + 64 * c2, a);
+                    ptx::tmem_ld32(tl + C::colS(x) + 64 * c2 + 32, b2);
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(a);
+                    ptx::reg_fence(b2);
+                    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) {
+                        float va = __uint_as_float(a[t]), vb = __uint_as_float(b2[t]);
+                        if (edge) {
+                            const int ca = 64 * c2 + t, cb = ca + 32;
+                            va = (ca >= cmin && ca <= cmax) ? va : -INFINITY;
+                            vb = (cb >= cmin && cb <= cmax) ? vb : -INFINITY;
+                        }
+                        m0 = fmaxf(m0, va);
+                        m1 = fmaxf(m1, vb);
+                    }
+                    mx = fmaxf(mx, fmaxf(m0, m1));
+                }
+                const float m_cand = mx * scale_log2;
+                bool need = false;
+                float alpha = 1.f;
+                if (m_cand > m_ref) {
+                    if (m_ref == -INFINITY) {
+                        m_ref = m_cand;  // first in-band keys of this row: O row and l are 0
+                    } else if (m_cand > m_ref + kPPRescaleThreshold) {
+                        need = true;
+                        alpha = ptx::ex2(m_ref - m_cand);
+                    }
+                }
+                if (__any_sync(0xffffffffu, need)) {
+                    // O_x holds exactly the tiles before kt (see the ordering note above)
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
+                        ptx::tmem_ld_wait();
+                        ptx::reg_fence(o);
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                        ptx::tmem_st32(tl + C::colO(x) + cc * 32, o);
+                    }
+                    ptx::tmem_st_wait();
+                    if (need) {
+                        l *= alpha;
+                        m_ref = m_cand;
+                    }
+                }
+                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+                // pass 2: P = exp2(s*c - m) packed as bf16 over the S columns already read
+                float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {  // chunk of 32 keys
+                    uint32_t a[32];
+                    ptx::tmem_ld32(tl + C::colS(x) + 32 * c, a);
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(a);
+                    uint32_t ph[16], pl[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        float v0 = __uint_as_float(a[2 * t]), v1 = __uint_as_float(a[2 * t + 1]);
+                        if (edge) {
+                            const int k0 = 32 * c + 2 * t;
+                            v0 = (k0 >= cmin && k0 <= cmax) ? v0 : -INFINITY;
+                            v1 = (k0 + 1 >= cmin && k0 + 1 <= cmax) ? v1 : -INFINITY;
+                        }
+                        const float e0 = ptx::ex2(fmaf(v0, scale_log2, -m_use));
+                        const float e1 = ptx::ex2(fmaf(v1, scale_log2, -m_use));
+                        ph[t] = ptx::pack_bf16x2_trunc(e0, e1);
+                        const float h0 = ptx::trunc_bf16(e0), h1 = ptx::trunc_bf16(e1);
+                        if (precise) {
+                            const float r0 = e0 - h0, r1 = e1 - h1;  // exact in fp32
+                            pl[t] = ptx::pack_bf16x2_trunc(r0, r1);
+                            ls0 += h0 + ptx::trunc_bf16(r0);
+                            ls1 += h1 + ptx::trunc_bf16(r1);
+                        } else {
+                            ls0 += h0;
+                            ls1 += h1;
+                        }
+                    }
+                    __syncwarp();
+                    ptx::tmem_st16(tl + C::colS(x) + 32 * c, ph);
+                    if (precise) ptx::tmem_st16(tl + C::colS(x) + 32 * c + 16, pl);
+                }
+                l += ls0 + ls1;
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(p_full + x);
+            }
+            if (!ok) break;
+            // ------------------------------------------------------------ epilogue
+            bool w = ptx::mbar_wait(o_final + x, ni & 1, wait_limit_ns, abort_flag);
+            ++ni;
+            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = out + ((int64_t)it.bh * T + i) * D;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
+                ptx::tmem_ld_wait();
+                ptx::reg_fence(o);
+                if (i < T) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        uint4 val;
+                        val.x = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 0]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l);
+                        val.y = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l);
+                        val.z = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l);
+                        val.w = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l);
+                        *reinterpret_cast<uint4*>(orow + cc * 32 + t * 8) = val;
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(o_free + x);  // O_x may be overwritten by the next item
+        }
+        if (!ok) {
+            atomicCAS(status, 0, 5);
+            *abort_flag = 1;
+        }
+    }
+
+    // -------------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        if (warp == 0 && lane == 0) {
+            // let every TMA load this CTA issued land before its shared memory goes away
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+                if (nq[x] > 0) ptx::mbar_wait(q_full + x, (nq[x] - 1) & 1, kPPDrainLimitNs, nullptr);
+            for (uint32_t st = 0; st < (uint32_t)NS && st < loads; ++st) {
+                const uint32_t t = st + ((loads - 1 - st) / NS) * NS;
+                ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);
+            }
+        }
+        if (warp == 1 && lane == 0) {
+            ptx::tc_commit(drain);  // completes when every MMA issued so far is done
+            ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace swa

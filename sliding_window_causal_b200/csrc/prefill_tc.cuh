@@ -69,6 +69,51 @@ __device__ __forceinline__ void record_status(int* status, int code) {
     atomicCAS(status, 0, code);
 }
 
+// P = exp2(s*c - m) for one 128-key row held by this thread, written to TMEM at column
+// col as bf16 pairs (rounded toward zero by a byte permute). PRECISE also writes the
+// remainder p - bf16(p), again as bf16, 64 columns further on. Returns the sum of the
+// weights exactly as written (so that O is normalised by the weights the MMAs used).
+template <bool PRECISE>
+__device__ __forceinline__ float write_p(const float (&sv)[128], float scale_log2, float m_use,
+                                         uint32_t col) {
+    float ls0 = 0.f, ls1 = 0.f;
+    if (!PRECISE) {
+        uint32_t p[2][32];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+            const float e0 = ptx::ex2(fmaf(sv[2 * c], scale_log2, -m_use));
+            const float e1 = ptx::ex2(fmaf(sv[2 * c + 1], scale_log2, -m_use));
+            p[c >> 5][c & 31] = ptx::pack_bf16x2_trunc(e0, e1);
+            ls0 += ptx::trunc_bf16(e0);
+            ls1 += ptx::trunc_bf16(e1);
+        }
+        __syncwarp();
+        ptx::tmem_st32(col, p[0]);
+        ptx::tmem_st32(col + 32, p[1]);
+    } else {
+        __syncwarp();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t ph[16], pl[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int cp = q4 * 16 + c;
+                const float e0 = ptx::ex2(fmaf(sv[2 * cp], scale_log2, -m_use));
+                const float e1 = ptx::ex2(fmaf(sv[2 * cp + 1], scale_log2, -m_use));
+                const float h0 = ptx::trunc_bf16(e0), h1 = ptx::trunc_bf16(e1);
+                const float r0 = e0 - h0, r1 = e1 - h1;  // exact in fp32
+                ph[c] = ptx::pack_bf16x2_trunc(e0, e1);
+                pl[c] = ptx::pack_bf16x2_trunc(r0, r1);
+                ls0 += h0 + ptx::trunc_bf16(r0);
+                ls1 += h1 + ptx::trunc_bf16(r1);
+            }
+            ptx::tmem_st16(col + q4 * 16, ph);
+            ptx::tmem_st16(col + 64 + q4 * 16, pl);
+        }
+    }
+    return ls0 + ls1;
+}
+
 template <int D, int NS>
 __global__ void __launch_bounds__(192, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -302,35 +347,8 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // P in chunks of 16 packed pairs (32 keys), each stored as soon as it is
-            // ready; the row sum counts exactly the bf16 weights the MMA multiplies by.
-            float ls0 = 0.f, ls1 = 0.f;
-            __syncwarp();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t ph[16], pl[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int cp = q4 * 16 + c;
-                    const float e0 = ptx::ex2(fmaf(sv[2 * cp], scale_log2, -m_use));
-                    const float e1 = ptx::ex2(fmaf(sv[2 * cp + 1], scale_log2, -m_use));
-                    const uint32_t hi = ptx::pack_bf16x2(e0, e1);
-                    const float h0 = ptx::bf16lo_f32(hi), h1 = ptx::bf16hi_f32(hi);
-                    ph[c] = hi;
-                    if (precise) {
-                        const uint32_t lo = ptx::pack_bf16x2(e0 - h0, e1 - h1);
-                        pl[c] = lo;
-                        ls0 += h0 + ptx::bf16lo_f32(lo);
-                        ls1 += h1 + ptx::bf16hi_f32(lo);
-                    } else {
-                        ls0 += h0;
-                        ls1 += h1;
-                    }
-                }
-                ptx::tmem_st16(tl + C::colS(b) + q4 * 16, ph);
-                if (precise) ptx::tmem_st16(tl + C::colS(b) + 64 + q4 * 16, pl);
-            }
-            l += ls0 + ls1;
+            l += precise ? write_p<true>(sv, scale_log2, m_use, tl + C::colS(b))
+                         : write_p<false>(sv, scale_log2, m_use, tl + C::colS(b));
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full + b);

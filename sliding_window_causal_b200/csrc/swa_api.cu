@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "plan.h"
 #include "prefill_simt.cuh"
+#include "prefill_pp.cuh"
 #include "prefill_tc.cuh"
 
 // Per-device status word: kernels record the first error here (atomicCAS from 0).
@@ -71,6 +72,7 @@ std::mutex g_mu;
 struct DeviceState {
     bool attrs_set = false;
     int* status = nullptr;  // device address of g_swa_status
+    int num_sms = 0;
 };
 std::map<int, DeviceState> g_dev;
 
@@ -95,6 +97,16 @@ int device_state(DeviceState** out) {
             e = cudaFuncSetAttribute(swa::prefill_tc_kernel<64, 4>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::TcCfg<64, 4>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<128>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::PPCfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::PPCfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::prefill_simt_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -271,6 +283,21 @@ int swa_forward(const void* q, const void* k, const void* v, void* out, int64_t 
             (rc = make_map(&mv, v, BH, T, D)) || (rc = make_map(&mo, out, BH, T, D)))
             return rc;
         const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+        const char* impl = getenv("SWA_PREFILL_IMPL");
+        if (!(impl && std::string(impl) == "tile")) {
+            const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
+            const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
+            auto* ob = static_cast<__nv_bfloat16*>(out);
+            if (D == 128)
+                swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
+                    mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
+            else
+                swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
+                    mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e, "swa_forward launch");
+            return success();
+        }
         const dim3 grid((unsigned)(n_qt * BH));
         if (D == 128) {
             swa::prefill_tc_kernel<128, 3><<<grid, 192, swa::TcCfg<128, 3>::kSmemBytes, s>>>(
