@@ -110,6 +110,90 @@ __device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W 
 // into 32c+16..32c+31), so that P only ever overwrites S values already read.
 __device__ __forceinline__ uint32_t pp_pcol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
+// Row maximum of the 128 scores this thread owns in the S buffer at TMEM column col;
+// on edge tiles the columns outside [cmin, cmax] count as -inf. The load of the next
+// 32-column chunk is in flight while the current one is reduced.
+template <bool EDGE>
+__device__ __forceinline__ float pp_rowmax(uint32_t col, int cmin, int cmax) {
+    uint32_t a[2][32];
+    float m0 = -INFINITY, m1 = -INFINITY;
+    ptx::tmem_ld32(col, a[0]);
+    ptx::tmem_ld_wait();
+    ptx::reg_fence(a[0]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (c + 1 < 4) ptx::tmem_ld32(col + 32 * (c + 1), a[(c + 1) & 1]);
+        const uint32_t(&v)[32] = a[c & 1];
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+            float v0 = __uint_as_float(v[t]), v1 = __uint_as_float(v[t + 1]);
+            float v2 = __uint_as_float(v[t + 2]), v3 = __uint_as_float(v[t + 3]);
+            if (EDGE) {
+                const int k = 32 * c + t;
+                v0 = (k >= cmin && k <= cmax) ? v0 : -INFINITY;
+                v1 = (k + 1 >= cmin && k + 1 <= cmax) ? v1 : -INFINITY;
+                v2 = (k + 2 >= cmin && k + 2 <= cmax) ? v2 : -INFINITY;
+                v3 = (k + 3 >= cmin && k + 3 <= cmax) ? v3 : -INFINITY;
+            }
+            m0 = ptx::max3(m0, v0, v1);
+            m1 = ptx::max3(m1, v2, v3);
+        }
+        if (c + 1 < 4) {
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(a[(c + 1) & 1]);
+        }
+    }
+    return fmaxf(m0, m1);
+}
+
+// P = exp2(s*c - m) for the 128 scores at TMEM column col, written back over them as
+// bf16 pairs (round to nearest): keys 32c..32c+31 go to columns 32c..32c+15 and, for
+// PRECISE tiles, the remainders p - bf16(p) (again bf16) to columns 32c+16..32c+31.
+// Returns the row sum of the unrounded weights (the rounding of P is unbiased, and for
+// PRECISE tiles hi + lo carries P to about 2^-17).
+template <bool EDGE, bool PRECISE>
+__device__ __forceinline__ float pp_exp_store(uint32_t col, float scale_log2, float m_use,
+                                              int cmin, int cmax) {
+    uint32_t a[2][32];
+    const ptx::f32x2 sc = {scale_log2, scale_log2}, nm = {-m_use, -m_use};
+    ptx::f32x2 acc0 = {0.f, 0.f}, acc1 = {0.f, 0.f};
+    ptx::tmem_ld32(col, a[0]);
+    ptx::tmem_ld_wait();
+    ptx::reg_fence(a[0]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (c + 1 < 4) ptx::tmem_ld32(col + 32 * (c + 1), a[(c + 1) & 1]);
+        const uint32_t(&v)[32] = a[c & 1];
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            ptx::f32x2 s2 = {__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])};
+            if (EDGE) {
+                const int k = 32 * c + 2 * t;
+                s2.x = (k >= cmin && k <= cmax) ? s2.x : -INFINITY;
+                s2.y = (k + 1 >= cmin && k + 1 <= cmax) ? s2.y : -INFINITY;
+            }
+            const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
+            const ptx::f32x2 e = {ptx::ex2(z.x), ptx::ex2(z.y)};
+            ph[t] = ptx::pack_bf16x2(e.x, e.y);
+            if (PRECISE) {
+                const ptx::f32x2 h = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
+                pl[t] = ptx::pack_bf16x2(e.x - h.x, e.y - h.y);
+            }
+            if (t & 1) acc1 = ptx::add2(acc1, e);
+            else acc0 = ptx::add2(acc0, e);
+        }
+        __syncwarp();
+        ptx::tmem_st16(col + 32 * c, ph);
+        if (PRECISE) ptx::tmem_st16(col + 32 * c + 16, pl);
+        if (c + 1 < 4) {
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(a[(c + 1) & 1]);
+        }
+    }
+    return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -327,29 +411,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool edge = tile_class(T, W, 128, 128, qt, kt) != 2;
                 const int cmin = lo - kt * 128, cmax = hi - kt * 128;
                 // pass 1: row max over the tile (masked on edge tiles)
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t a[32], b2[32];
-                    ptx::tmem_ld32(tl + C::colS(x) + 64 * c2, a);
-                    ptx::tmem_ld32(tl + C::colS(x) + 64 * c2 + 32, b2);
-                    ptx::tmem_ld_wait();
-                    ptx::reg_fence(a);
-                    ptx::reg_fence(b2);
-                    float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-                    for (int t = 0; t < 32; ++t) {
-                        float va = __uint_as_float(a[t]), vb = __uint_as_float(b2[t]);
-                        if (edge) {
-                            const int ca = 64 * c2 + t, cb = ca + 32;
-                            va = (ca >= cmin && ca <= cmax) ? va : -INFINITY;
-                            vb = (cb >= cmin && cb <= cmax) ? vb : -INFINITY;
-                        }
-                        m0 = fmaxf(m0, va);
-                        m1 = fmaxf(m1, vb);
-                    }
-                    mx = fmaxf(mx, fmaxf(m0, m1));
-                }
+                const float mx = edge ? pp_rowmax<true>(tl + C::colS(x), cmin, cmax)
+                                      : pp_rowmax<false>(tl + C::colS(x), cmin, cmax);
                 const float m_cand = mx * scale_log2;
                 bool need = false;
                 float alpha = 1.f;
@@ -381,41 +444,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 }
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
                 // pass 2: P = exp2(s*c - m) packed as bf16 over the S columns already read
-                float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {  // chunk of 32 keys
-                    uint32_t a[32];
-                    ptx::tmem_ld32(tl + C::colS(x) + 32 * c, a);
-                    ptx::tmem_ld_wait();
-                    ptx::reg_fence(a);
-                    uint32_t ph[16], pl[16];
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        float v0 = __uint_as_float(a[2 * t]), v1 = __uint_as_float(a[2 * t + 1]);
-                        if (edge) {
-                            const int k0 = 32 * c + 2 * t;
-                            v0 = (k0 >= cmin && k0 <= cmax) ? v0 : -INFINITY;
-                            v1 = (k0 + 1 >= cmin && k0 + 1 <= cmax) ? v1 : -INFINITY;
-                        }
-                        const float e0 = ptx::ex2(fmaf(v0, scale_log2, -m_use));
-                        const float e1 = ptx::ex2(fmaf(v1, scale_log2, -m_use));
-                        ph[t] = ptx::pack_bf16x2_trunc(e0, e1);
-                        const float h0 = ptx::trunc_bf16(e0), h1 = ptx::trunc_bf16(e1);
-                        if (precise) {
-                            const float r0 = e0 - h0, r1 = e1 - h1;  // exact in fp32
-                            pl[t] = ptx::pack_bf16x2_trunc(r0, r1);
-                            ls0 += h0 + ptx::trunc_bf16(r0);
-                            ls1 += h1 + ptx::trunc_bf16(r1);
-                        } else {
-                            ls0 += h0;
-                            ls1 += h1;
-                        }
-                    }
-                    __syncwarp();
-                    ptx::tmem_st16(tl + C::colS(x) + 32 * c, ph);
-                    if (precise) ptx::tmem_st16(tl + C::colS(x) + 32 * c + 16, pl);
-                }
-                l += ls0 + ls1;
+                const uint32_t scol = tl + C::colS(x);
+                float ls;
+                if (edge) ls = precise ? pp_exp_store<true, true>(scol, scale_log2, m_use, cmin, cmax)
+                                       : pp_exp_store<true, false>(scol, scale_log2, m_use, cmin, cmax);
+                else ls = precise ? pp_exp_store<false, true>(scol, scale_log2, m_use, cmin, cmax)
+                                  : pp_exp_store<false, false>(scol, scale_log2, m_use, cmin, cmax);
+                l += ls;
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_full + x);
