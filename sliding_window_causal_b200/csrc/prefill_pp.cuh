@@ -194,6 +194,115 @@ __device__ __forceinline__ float pp_exp_store(uint32_t col, float scale_log2, fl
     return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
 
+// 2^-k for an integer k in [0, 126], exactly.
+__device__ __forceinline__ float pp_pow2_neg(int k) { return __uint_as_float((uint32_t)(127 - k) << 23); }
+
+// Multiply this thread's O row (D fp32 columns at TMEM column ocol) by a, and the bf16 P
+// already written for the first `chunks` 32-key chunks of the S buffer at scol (and
+// their low parts when PRECISE) by the same a. Warp-collective; a = 1 leaves a row as is.
+// With a a power of two the products are exact (barring underflow to zero).
+template <int D, bool PRECISE>
+__device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chunks, float a) {
+    ptx::tmem_st_wait();  // the P chunks read back below were written by this thread
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld32(ocol + cc * 32, o);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(o);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * a);
+        ptx::tmem_st32(ocol + cc * 32, o);
+    }
+#pragma unroll 1
+    for (int c = 0; c < chunks; ++c) {
+#pragma unroll
+        for (int part = 0; part < (PRECISE ? 2 : 1); ++part) {
+            uint32_t p[16];
+            ptx::tmem_ld16(scol + 32 * c + 16 * part, p);
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(p);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                p[t] = ptx::pack_bf16x2(ptx::bf16lo_f32(p[t]) * a, ptx::bf16hi_f32(p[t]) * a);
+            ptx::tmem_st16(scol + 32 * c + 16 * part, p);
+        }
+    }
+    ptx::tmem_st_wait();
+}
+
+// One pass over a tile whose rows all have a finite reference m (log2 units): P =
+// exp2(s*c - m) is written chunk by chunk over the S columns (layout as pp_exp_store)
+// while each chunk's maximum is checked. When a row's chunk maximum exceeds m by more
+// than the rescale threshold, m moves up by the integer k = ceil(excess) and O, the P
+// already written for this tile and l are scaled by 2^-k (exactly) before the chunk is
+// recomputed. Returns the row-sum contribution of the tile; m and l are updated in place.
+template <int D, bool EDGE, bool PRECISE>
+__device__ __forceinline__ float pp_exp_store_1pass(uint32_t scol, uint32_t ocol, float scale_log2,
+                                                    float& m, float& l, int cmin, int cmax) {
+    uint32_t a[2][32];
+    const ptx::f32x2 sc = {scale_log2, scale_log2};
+    ptx::f32x2 acc0 = {0.f, 0.f}, acc1 = {0.f, 0.f};
+    ptx::tmem_ld32(scol, a[0]);
+    ptx::tmem_ld_wait();
+    ptx::reg_fence(a[0]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (c + 1 < 4) ptx::tmem_ld32(scol + 32 * (c + 1), a[(c + 1) & 1]);
+        uint32_t(&v)[32] = a[c & 1];
+        if (EDGE) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int k = 32 * c + t;
+                if (!(k >= cmin && k <= cmax)) v[t] = __float_as_uint(-INFINITY);
+            }
+        }
+        float q0 = -INFINITY, q1 = -INFINITY, q2 = -INFINITY, q3 = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < 32; t += 8) {
+            q0 = ptx::max3(q0, __uint_as_float(v[t]), __uint_as_float(v[t + 1]));
+            q1 = ptx::max3(q1, __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3]));
+            q2 = ptx::max3(q2, __uint_as_float(v[t + 4]), __uint_as_float(v[t + 5]));
+            q3 = ptx::max3(q3, __uint_as_float(v[t + 6]), __uint_as_float(v[t + 7]));
+        }
+        const float cm = fmaxf(fmaxf(q0, q1), fmaxf(q2, q3)) * scale_log2;
+        const bool need = cm > m + kPPRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+            int k = 0;
+            if (need) k = min(126, (int)ceilf(cm - m));
+            const float f = pp_pow2_neg(k);
+            __syncwarp();
+            pp_rescale<D, PRECISE>(ocol, scol, c, f);
+            l *= f;
+            acc0.x *= f; acc0.y *= f; acc1.x *= f; acc1.y *= f;
+            m += (float)k;
+        }
+        const ptx::f32x2 nm = {-m, -m};
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const ptx::f32x2 s2 = {__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])};
+            const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
+            const ptx::f32x2 e = {ptx::ex2(z.x), ptx::ex2(z.y)};
+            ph[t] = ptx::pack_bf16x2(e.x, e.y);
+            if (PRECISE) {
+                const ptx::f32x2 h = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
+                pl[t] = ptx::pack_bf16x2(e.x - h.x, e.y - h.y);
+            }
+            if (t & 1) acc1 = ptx::add2(acc1, e);
+            else acc0 = ptx::add2(acc0, e);
+        }
+        __syncwarp();
+        ptx::tmem_st16(scol + 32 * c, ph);
+        if (PRECISE) ptx::tmem_st16(scol + 32 * c + 16, pl);
+        if (c + 1 < 4) {
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(a[(c + 1) & 1]);
+        }
+    }
+    return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -410,46 +519,54 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 ptx::tc_fence_after();
                 const bool edge = tile_class(T, W, 128, 128, qt, kt) != 2;
                 const int cmin = lo - kt * 128, cmax = hi - kt * 128;
-                // pass 1: row max over the tile (masked on edge tiles)
-                const float mx = edge ? pp_rowmax<true>(tl + C::colS(x), cmin, cmax)
-                                      : pp_rowmax<false>(tl + C::colS(x), cmin, cmax);
-                const float m_cand = mx * scale_log2;
-                bool need = false;
-                float alpha = 1.f;
-                if (m_cand > m_ref) {
-                    if (m_ref == -INFINITY) {
-                        m_ref = m_cand;  // first in-band keys of this row: O row and l are 0
-                    } else if (m_cand > m_ref + kPPRescaleThreshold) {
-                        need = true;
-                        alpha = ptx::ex2(m_ref - m_cand);
-                    }
-                }
-                if (__any_sync(0xffffffffu, need)) {
-                    // O_x holds exactly the tiles before kt (see the ordering note above)
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
-                        ptx::tmem_ld_wait();
-                        ptx::reg_fence(o);
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                        ptx::tmem_st32(tl + C::colO(x) + cc * 32, o);
-                    }
-                    ptx::tmem_st_wait();
-                    if (need) {
-                        l *= alpha;
-                        m_ref = m_cand;
-                    }
-                }
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                // pass 2: P = exp2(s*c - m) packed as bf16 over the S columns already read
-                const uint32_t scol = tl + C::colS(x);
+                const uint32_t scol = tl + C::colS(x), ocol = tl + C::colO(x);
                 float ls;
-                if (edge) ls = precise ? pp_exp_store<true, true>(scol, scale_log2, m_use, cmin, cmax)
-                                       : pp_exp_store<true, false>(scol, scale_log2, m_use, cmin, cmax);
-                else ls = precise ? pp_exp_store<false, true>(scol, scale_log2, m_use, cmin, cmax)
-                                  : pp_exp_store<false, false>(scol, scale_log2, m_use, cmin, cmax);
+                if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+                    // steady state: one pass, the reference max moves only when it must
+                    if (edge) ls = precise ? pp_exp_store_1pass<D, true, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax)
+                                           : pp_exp_store_1pass<D, true, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                    else ls = precise ? pp_exp_store_1pass<D, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax)
+                                      : pp_exp_store_1pass<D, false, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                } else {
+                    // pass 1: row max over the tile (masked on edge tiles)
+                    const float mx = edge ? pp_rowmax<true>(tl + C::colS(x), cmin, cmax)
+                                          : pp_rowmax<false>(tl + C::colS(x), cmin, cmax);
+                    const float m_cand = mx * scale_log2;
+                    bool need = false;
+                    float alpha = 1.f;
+                    if (m_cand > m_ref) {
+                        if (m_ref == -INFINITY) {
+                            m_ref = m_cand;  // first in-band keys of this row: O row and l are 0
+                        } else if (m_cand > m_ref + kPPRescaleThreshold) {
+                            need = true;
+                            alpha = ptx::ex2(m_ref - m_cand);
+                        }
+                    }
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O_x holds exactly the tiles before kt (see the ordering note above)
+#pragma unroll 1
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t o[32];
+                            ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
+                            ptx::tmem_ld_wait();
+                            ptx::reg_fence(o);
+#pragma unroll
+                            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                            ptx::tmem_st32(tl + C::colO(x) + cc * 32, o);
+                        }
+                        ptx::tmem_st_wait();
+                        if (need) {
+                            l *= alpha;
+                            m_ref = m_cand;
+                        }
+                    }
+                    const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+                    // pass 2: P = exp2(s*c - m) packed as bf16 over the S columns already read
+                    if (edge) ls = precise ? pp_exp_store<true, true>(scol, scale_log2, m_use, cmin, cmax)
+                                           : pp_exp_store<true, false>(scol, scale_log2, m_use, cmin, cmax);
+                    else ls = precise ? pp_exp_store<false, true>(scol, scale_log2, m_use, cmin, cmax)
+                                      : pp_exp_store<false, false>(scol, scale_log2, m_use, cmin, cmax);
+                }
                 l += ls;
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();

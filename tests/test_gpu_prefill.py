@@ -200,3 +200,20 @@ def test_mistral_shaped_sampled():
 @pytest.mark.parametrize("wl", inputs.SWEEP, ids=lambda w: w.name)
 def test_window_sweep_sampled(wl):
     sampled_parity(wl, [(0, 0), (1, 15)], n_random=48)
+
+
+@pytest.mark.parametrize("D,W", [(128, 4096), (64, 700), (128, 200)])
+def test_growing_scores_move_the_reference(D, W):
+    """Scores that grow steadily along the sequence (q . k_j grows with j) push every
+    row's running maximum up by far more than the lazy-rescale threshold, tile after
+    tile and chunk after chunk inside a tile; the output must still match."""
+    T = 1500
+    gen = torch.Generator().manual_seed(71)
+    q = torch.ones(1, 2, T, D)
+    k = (torch.arange(T, dtype=torch.float32) * 0.05)[None, None, :, None].expand(1, 2, T, D).clone()
+    k += 0.01 * torch.randn(1, 2, T, D, generator=gen)
+    v = torch.randn(1, 2, T, D, generator=gen)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    out = run(q, k, v, W)
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    assert max_err(out, ref) <= TOL[torch.bfloat16]
