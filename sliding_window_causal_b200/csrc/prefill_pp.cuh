@@ -110,90 +110,6 @@ __device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W 
 // into 32c+16..32c+31), so that P only ever overwrites S values already read.
 __device__ __forceinline__ uint32_t pp_pcol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
-// Row maximum of the 128 scores this thread owns in the S buffer at TMEM column col;
-// on edge tiles the columns outside [cmin, cmax] count as -inf. The load of the next
-// 32-column chunk is in flight while the current one is reduced.
-template <bool EDGE>
-__device__ __forceinline__ float pp_rowmax(uint32_t col, int cmin, int cmax) {
-    uint32_t a[2][32];
-    float m0 = -INFINITY, m1 = -INFINITY;
-    ptx::tmem_ld32(col, a[0]);
-    ptx::tmem_ld_wait();
-    ptx::reg_fence(a[0]);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        if (c + 1 < 4) ptx::tmem_ld32(col + 32 * (c + 1), a[(c + 1) & 1]);
-        const uint32_t(&v)[32] = a[c & 1];
-#pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-            float v0 = __uint_as_float(v[t]), v1 = __uint_as_float(v[t + 1]);
-            float v2 = __uint_as_float(v[t + 2]), v3 = __uint_as_float(v[t + 3]);
-            if (EDGE) {
-                const int k = 32 * c + t;
-                v0 = (k >= cmin && k <= cmax) ? v0 : -INFINITY;
-                v1 = (k + 1 >= cmin && k + 1 <= cmax) ? v1 : -INFINITY;
-                v2 = (k + 2 >= cmin && k + 2 <= cmax) ? v2 : -INFINITY;
-                v3 = (k + 3 >= cmin && k + 3 <= cmax) ? v3 : -INFINITY;
-            }
-            m0 = ptx::max3(m0, v0, v1);
-            m1 = ptx::max3(m1, v2, v3);
-        }
-        if (c + 1 < 4) {
-            ptx::tmem_ld_wait();
-            ptx::reg_fence(a[(c + 1) & 1]);
-        }
-    }
-    return fmaxf(m0, m1);
-}
-
-// P = exp2(s*c - m) for the 128 scores at TMEM column col, written back over them as
-// bf16 pairs (round to nearest): keys 32c..32c+31 go to columns 32c..32c+15 and, for
-// PRECISE tiles, the remainders p - bf16(p) (again bf16) to columns 32c+16..32c+31.
-// Returns the row sum of the unrounded weights (the rounding of P is unbiased, and for
-// PRECISE tiles hi + lo carries P to about 2^-17).
-template <bool EDGE, bool PRECISE>
-__device__ __forceinline__ float pp_exp_store(uint32_t col, float scale_log2, float m_use,
-                                              int cmin, int cmax) {
-    uint32_t a[2][32];
-    const ptx::f32x2 sc = {scale_log2, scale_log2}, nm = {-m_use, -m_use};
-    ptx::f32x2 acc0 = {0.f, 0.f}, acc1 = {0.f, 0.f};
-    ptx::tmem_ld32(col, a[0]);
-    ptx::tmem_ld_wait();
-    ptx::reg_fence(a[0]);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        if (c + 1 < 4) ptx::tmem_ld32(col + 32 * (c + 1), a[(c + 1) & 1]);
-        const uint32_t(&v)[32] = a[c & 1];
-        uint32_t ph[16], pl[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            ptx::f32x2 s2 = {__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])};
-            if (EDGE) {
-                const int k = 32 * c + 2 * t;
-                s2.x = (k >= cmin && k <= cmax) ? s2.x : -INFINITY;
-                s2.y = (k + 1 >= cmin && k + 1 <= cmax) ? s2.y : -INFINITY;
-            }
-            const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
-            const ptx::f32x2 e = {ptx::ex2(z.x), ptx::ex2(z.y)};
-            ph[t] = ptx::pack_bf16x2(e.x, e.y);
-            if (PRECISE) {
-                const ptx::f32x2 h = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
-                pl[t] = ptx::pack_bf16x2(e.x - h.x, e.y - h.y);
-            }
-            if (t & 1) acc1 = ptx::add2(acc1, e);
-            else acc0 = ptx::add2(acc0, e);
-        }
-        __syncwarp();
-        ptx::tmem_st16(col + 32 * c, ph);
-        if (PRECISE) ptx::tmem_st16(col + 32 * c + 16, pl);
-        if (c + 1 < 4) {
-            ptx::tmem_ld_wait();
-            ptx::reg_fence(a[(c + 1) & 1]);
-        }
-    }
-    return (acc0.x + acc0.y) + (acc1.x + acc1.y);
-}
-
 // 2^-k for an integer k in [0, 126], exactly.
 __device__ __forceinline__ float pp_pow2_neg(int k) { return __uint_as_float((uint32_t)(127 - k) << 23); }
 
@@ -231,18 +147,22 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
     ptx::tmem_st_wait();
 }
 
-// One pass over a tile whose rows all have a finite reference m (log2 units): P =
-// exp2(s*c - m) is written chunk by chunk over the S columns (layout as pp_exp_store)
-// while each chunk's maximum is checked. When a row's chunk maximum exceeds m by more
-// than the rescale threshold, m moves up by the integer k = ceil(excess) and O, the P
-// already written for this tile and l are scaled by 2^-k (exactly) before the chunk is
-// recomputed. Returns the row-sum contribution of the tile; m and l are updated in place.
+// One pass over a tile: P = exp2(s*c - m) is written chunk by chunk (32 keys) over the
+// S columns of the tile, keys 32c..32c+31 packed as bf16 pairs (round to nearest) into
+// columns 32c..32c+15 and, for PRECISE tiles, the remainders p - bf16(p) (again bf16)
+// into columns 32c+16..32c+31, so that P only overwrites S values already read.
+// m is the row's reference maximum in log2 units (-inf until the row meets its first
+// in-band key). Each chunk's maximum is checked first: a row that sees its first keys
+// takes the chunk maximum as m; a row whose maximum exceeds m by more than the rescale
+// threshold moves m up by the integer k = ceil(excess), and O, the P already written
+// for this tile and l are scaled by 2^-k, which is exact. The row sum adds the weights
+// exactly as written, so O is normalised by the weights the MMAs multiply by.
 template <int D, bool EDGE, bool PRECISE>
-__device__ __forceinline__ float pp_exp_store_1pass(uint32_t scol, uint32_t ocol, float scale_log2,
-                                                    float& m, float& l, int cmin, int cmax) {
+__device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
+                                        float& l, int cmin, int cmax) {
     uint32_t a[2][32];
     const ptx::f32x2 sc = {scale_log2, scale_log2};
-    ptx::f32x2 acc0 = {0.f, 0.f}, acc1 = {0.f, 0.f};
+    ptx::f32x2 acc = {0.f, 0.f};
     ptx::tmem_ld32(scol, a[0]);
     ptx::tmem_ld_wait();
     ptx::reg_fence(a[0]);
@@ -266,31 +186,33 @@ __device__ __forceinline__ float pp_exp_store_1pass(uint32_t scol, uint32_t ocol
             q3 = ptx::max3(q3, __uint_as_float(v[t + 6]), __uint_as_float(v[t + 7]));
         }
         const float cm = fmaxf(fmaxf(q0, q1), fmaxf(q2, q3)) * scale_log2;
-        const bool need = cm > m + kPPRescaleThreshold;
+        const bool need = m != -INFINITY && cm > m + kPPRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
-            int k = 0;
-            if (need) k = min(126, (int)ceilf(cm - m));
+            const int k = need ? min(126, (int)ceilf(cm - m)) : 0;
             const float f = pp_pow2_neg(k);
             __syncwarp();
             pp_rescale<D, PRECISE>(ocol, scol, c, f);
             l *= f;
-            acc0.x *= f; acc0.y *= f; acc1.x *= f; acc1.y *= f;
+            acc.x *= f;
+            acc.y *= f;
             m += (float)k;
         }
-        const ptx::f32x2 nm = {-m, -m};
+        if (m == -INFINITY) m = cm;  // first in-band keys of the row (or still none)
+        const float mu = m == -INFINITY ? 0.f : m;
+        const ptx::f32x2 nm = {-mu, -mu};
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
             const ptx::f32x2 s2 = {__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])};
             const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
-            const ptx::f32x2 e = {ptx::ex2(z.x), ptx::ex2(z.y)};
-            ph[t] = ptx::pack_bf16x2(e.x, e.y);
+            const float e0 = ptx::ex2(z.x), e1 = ptx::ex2(z.y);
+            ph[t] = ptx::pack_bf16x2(e0, e1);
+            ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
             if (PRECISE) {
-                const ptx::f32x2 h = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
-                pl[t] = ptx::pack_bf16x2(e.x - h.x, e.y - h.y);
+                pl[t] = ptx::pack_bf16x2(e0 - w.x, e1 - w.y);
+                acc = ptx::add2(acc, {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
             }
-            if (t & 1) acc1 = ptx::add2(acc1, e);
-            else acc0 = ptx::add2(acc0, e);
+            acc = ptx::add2(acc, w);
         }
         __syncwarp();
         ptx::tmem_st16(scol + 32 * c, ph);
@@ -300,7 +222,7 @@ __device__ __forceinline__ float pp_exp_store_1pass(uint32_t scol, uint32_t ocol
             ptx::reg_fence(a[(c + 1) & 1]);
         }
     }
-    return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+    l += acc.x + acc.y;
 }
 
 template <int D>
@@ -520,54 +442,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool edge = tile_class(T, W, 128, 128, qt, kt) != 2;
                 const int cmin = lo - kt * 128, cmax = hi - kt * 128;
                 const uint32_t scol = tl + C::colS(x), ocol = tl + C::colO(x);
-                float ls;
-                if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
-                    // steady state: one pass, the reference max moves only when it must
-                    if (edge) ls = precise ? pp_exp_store_1pass<D, true, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax)
-                                           : pp_exp_store_1pass<D, true, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
-                    else ls = precise ? pp_exp_store_1pass<D, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax)
-                                      : pp_exp_store_1pass<D, false, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                if (edge) {
+                    if (precise) pp_tile<D, true, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                    else pp_tile<D, true, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
                 } else {
-                    // pass 1: row max over the tile (masked on edge tiles)
-                    const float mx = edge ? pp_rowmax<true>(tl + C::colS(x), cmin, cmax)
-                                          : pp_rowmax<false>(tl + C::colS(x), cmin, cmax);
-                    const float m_cand = mx * scale_log2;
-                    bool need = false;
-                    float alpha = 1.f;
-                    if (m_cand > m_ref) {
-                        if (m_ref == -INFINITY) {
-                            m_ref = m_cand;  // first in-band keys of this row: O row and l are 0
-                        } else if (m_cand > m_ref + kPPRescaleThreshold) {
-                            need = true;
-                            alpha = ptx::ex2(m_ref - m_cand);
-                        }
-                    }
-                    if (__any_sync(0xffffffffu, need)) {
-                        // O_x holds exactly the tiles before kt (see the ordering note above)
-#pragma unroll 1
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t o[32];
-                            ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
-                            ptx::tmem_ld_wait();
-                            ptx::reg_fence(o);
-#pragma unroll
-                            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                            ptx::tmem_st32(tl + C::colO(x) + cc * 32, o);
-                        }
-                        ptx::tmem_st_wait();
-                        if (need) {
-                            l *= alpha;
-                            m_ref = m_cand;
-                        }
-                    }
-                    const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                    // pass 2: P = exp2(s*c - m) packed as bf16 over the S columns already read
-                    if (edge) ls = precise ? pp_exp_store<true, true>(scol, scale_log2, m_use, cmin, cmax)
-                                           : pp_exp_store<true, false>(scol, scale_log2, m_use, cmin, cmax);
-                    else ls = precise ? pp_exp_store<false, true>(scol, scale_log2, m_use, cmin, cmax)
-                                      : pp_exp_store<false, false>(scol, scale_log2, m_use, cmin, cmax);
+                    if (precise) pp_tile<D, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                    else pp_tile<D, false, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
                 }
-                l += ls;
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_full + x);
