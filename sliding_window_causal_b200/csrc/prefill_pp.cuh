@@ -11,7 +11,7 @@
 // of the list ordered heaviest first (a snake over the list), which balances the load
 // without any device-side queue.
 //
-// Roles (320 threads, one CTA per SM):
+// Roles (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0, lane 0     TMA producer: Q_A, Q_B per item, then K_kt and V_kt through one
 //                      NSTAGE-deep ring of 128-row tiles.
 //   warp 1             allocates the 512 TMEM columns; lane 0 issues every tcgen05 MMA in
@@ -19,7 +19,7 @@
 //                      core works on one tile's products while the other tile's softmax runs:
 //                        S_X = Q_X K^T   -> TMEM columns [128X, 128X+128)   (fp32)
 //                        O_X += P_X V    -> TMEM columns [256+128X, +D)     (fp32)
-//   warps 2..5 (A), 6..9 (B)    softmax of one query tile each, one row per thread (warp w
+//   warps 4..7 (A), 8..11 (B)   softmax of one query tile each, one row per thread (warp w
 //                      reads TMEM lanes 32*(w%4)..): running max and sum of the online
 //                      softmax ("Mistral Architecture > Implementation: Sliding Window
 //                      Attention", Step 2, stable softmax), -inf select on edge tiles, P
@@ -41,7 +41,16 @@
 
 namespace swa {
 
-constexpr int kPPThreads = 320;
+constexpr int kPPThreads = 384;
+// Register split (setmaxnreg): the CTA is launched with kPPLaunchRegs per thread
+// (384 x 168 = 64512); the producer/MMA warpgroup gives registers back down to
+// kPPRoleRegs and the two softmax warpgroups take them up to kPPSoftmaxRegs:
+// 128 x 96 + 256 x 200 = 63488 <= 64512. The host refuses to launch if the compiled kernel does
+// not use exactly kPPLaunchRegs (an increase the pool cannot cover would never return).
+constexpr int kPPLaunchRegs = 168;
+constexpr int kPPRoleRegs = 96;
+constexpr int kPPSoftmaxRegs = 200;
+static_assert(128 * kPPRoleRegs + 256 * kPPSoftmaxRegs <= kPPThreads * kPPLaunchRegs, "register split");
 constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow by 2^8 first
 // Query tiles whose rows see few keys (the first tile of every head, or any tile when
 // W <= kPPPreciseWindow) carry P as two bf16 parts hi + lo with a second P.V MMA: there a
@@ -147,82 +156,77 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
     ptx::tmem_st_wait();
 }
 
-// One pass over a tile: P = exp2(s*c - m) is written chunk by chunk (32 keys) over the
-// S columns of the tile, keys 32c..32c+31 packed as bf16 pairs (round to nearest) into
-// columns 32c..32c+15 and, for PRECISE tiles, the remainders p - bf16(p) (again bf16)
-// into columns 32c+16..32c+31, so that P only overwrites S values already read.
-// m is the row's reference maximum in log2 units (-inf until the row meets its first
-// in-band key). Each chunk's maximum is checked first: a row that sees its first keys
-// takes the chunk maximum as m; a row whose maximum exceeds m by more than the rescale
-// threshold moves m up by the integer k = ceil(excess), and O, the P already written
-// for this tile and l are scaled by 2^-k, which is exact. The row sum adds the weights
-// exactly as written, so O is normalised by the weights the MMAs multiply by.
+// One tile of one row: the thread's 128 scores are read from TMEM in one round trip,
+// masked on edge tiles, reduced to the row maximum (log2 units), and P = exp2(s*c - m)
+// is written back over the S columns as bf16 pairs (round to nearest): keys 32c..32c+31
+// into columns 32c..32c+15 and, for PRECISE tiles, the remainders p - bf16(p) (again
+// bf16) into columns 32c+16..32c+31.
+// m is the row's reference maximum (-inf until the row meets its first in-band key). A
+// row that sees its first keys takes the tile maximum; a row whose maximum exceeds m by
+// more than the rescale threshold moves m up by the integer k = ceil(excess) and scales
+// O and l by 2^-k (exact). The row sum adds the weights exactly as written, so O is
+// normalised by the weights the MMAs multiply by.
 template <int D, bool EDGE, bool PRECISE>
 __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
                                         float& l, int cmin, int cmax) {
-    uint32_t a[2][32];
-    const ptx::f32x2 sc = {scale_log2, scale_log2};
-    ptx::f32x2 acc = {0.f, 0.f};
-    ptx::tmem_ld32(scol, a[0]);
-    ptx::tmem_ld_wait();
-    ptx::reg_fence(a[0]);
+    uint32_t v[4][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        if (c + 1 < 4) ptx::tmem_ld32(scol + 32 * (c + 1), a[(c + 1) & 1]);
-        uint32_t(&v)[32] = a[c & 1];
-        if (EDGE) {
+    for (int c = 0; c < 4; ++c) ptx::tmem_ld32(scol + 32 * c, v[c]);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ptx::reg_fence(v[c]);
+    if (EDGE) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int k = 32 * c + t;
-                if (!(k >= cmin && k <= cmax)) v[t] = __float_as_uint(-INFINITY);
+                if (!(k >= cmin && k <= cmax)) v[c][t] = __float_as_uint(-INFINITY);
             }
-        }
-        float q0 = -INFINITY, q1 = -INFINITY, q2 = -INFINITY, q3 = -INFINITY;
+    }
+    float q[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int t = 0; t < 32; t += 8) {
-            q0 = ptx::max3(q0, __uint_as_float(v[t]), __uint_as_float(v[t + 1]));
-            q1 = ptx::max3(q1, __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3]));
-            q2 = ptx::max3(q2, __uint_as_float(v[t + 4]), __uint_as_float(v[t + 5]));
-            q3 = ptx::max3(q3, __uint_as_float(v[t + 6]), __uint_as_float(v[t + 7]));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                q[j] = ptx::max3(q[j], __uint_as_float(v[c][t + 2 * j]), __uint_as_float(v[c][t + 2 * j + 1]));
         }
-        const float cm = fmaxf(fmaxf(q0, q1), fmaxf(q2, q3)) * scale_log2;
-        const bool need = m != -INFINITY && cm > m + kPPRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-            const int k = need ? min(126, (int)ceilf(cm - m)) : 0;
-            const float f = pp_pow2_neg(k);
-            __syncwarp();
-            pp_rescale<D, PRECISE>(ocol, scol, c, f);
-            l *= f;
-            acc.x *= f;
-            acc.y *= f;
-            m += (float)k;
-        }
-        if (m == -INFINITY) m = cm;  // first in-band keys of the row (or still none)
-        const float mu = m == -INFINITY ? 0.f : m;
-        const ptx::f32x2 nm = {-mu, -mu};
+    const float tm = fmaxf(fmaxf(q[0], q[1]), fmaxf(q[2], q[3])) * scale_log2;
+    const bool need = m != -INFINITY && tm > m + kPPRescaleThreshold;
+    if (__any_sync(0xffffffffu, need)) {
+        const int k = need ? min(126, (int)ceilf(tm - m)) : 0;
+        const float f = pp_pow2_neg(k);
+        __syncwarp();
+        pp_rescale<D, PRECISE>(ocol, scol, 0, f);
+        l *= f;
+        m += (float)k;
+    }
+    if (m == -INFINITY) m = tm;  // first in-band keys of the row (or still none)
+    const float mu = m == -INFINITY ? 0.f : m;
+    const ptx::f32x2 sc = {scale_log2, scale_log2}, nm = {-mu, -mu};
+    ptx::f32x2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-            const ptx::f32x2 s2 = {__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])};
+            const ptx::f32x2 s2 = {__uint_as_float(v[c][2 * t]), __uint_as_float(v[c][2 * t + 1])};
             const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
             const float e0 = ptx::ex2(z.x), e1 = ptx::ex2(z.y);
             ph[t] = ptx::pack_bf16x2(e0, e1);
-            ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
+            const ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
             if (PRECISE) {
                 pl[t] = ptx::pack_bf16x2(e0 - w.x, e1 - w.y);
-                acc = ptx::add2(acc, {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
+                acc[(t + 2) & 3] = ptx::add2(acc[(t + 2) & 3], {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
             }
-            acc = ptx::add2(acc, w);
+            acc[t & 3] = ptx::add2(acc[t & 3], w);
         }
-        __syncwarp();
         ptx::tmem_st16(scol + 32 * c, ph);
         if (PRECISE) ptx::tmem_st16(scol + 32 * c + 16, pl);
-        if (c + 1 < 4) {
-            ptx::tmem_ld_wait();
-            ptx::reg_fence(a[(c + 1) & 1]);
-        }
     }
-    l += acc.x + acc.y;
+    l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
 template <int D>
@@ -287,7 +291,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     uint32_t loads = 0;  // producer: K/V tiles issued so far
     int nq[2] = {0, 0};  // producer: Q tiles issued per side
 
-    if (warp == 0) {
+    if (warp < 4) {
+      ptx::regs_dec<kPPRoleRegs>();
+      if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ producer
             bool ok = true;
@@ -411,9 +417,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 *abort_flag = 1;
             }
         }
+      }
     } else {
+        ptx::regs_inc<kPPSoftmaxRegs>();
         // ---------------------------------------------------------------- softmax A / B
-        const int x = (warp - 2) >> 2;   // 0: tile A, 1: tile B
+        const int x = (warp - 4) >> 2;   // 0: tile A, 1: tile B
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);

@@ -73,6 +73,7 @@ struct DeviceState {
     bool attrs_set = false;
     int* status = nullptr;  // device address of g_swa_status
     int num_sms = 0;
+    bool pp_regs_ok = false;  // the persistent prefill kernels use exactly kPPLaunchRegs
 };
 std::map<int, DeviceState> g_dev;
 
@@ -107,6 +108,14 @@ int device_state(DeviceState** out) {
                                      swa::PPCfg<64>::kSmemBytes);
         if (e == cudaSuccess)
             e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) {
+            // The register split inside the kernel assumes this launch allocation.
+            cudaFuncAttributes a128, a64;
+            e = cudaFuncGetAttributes(&a128, swa::prefill_pp_kernel<128>);
+            if (e == cudaSuccess) e = cudaFuncGetAttributes(&a64, swa::prefill_pp_kernel<64>);
+            st.pp_regs_ok = e == cudaSuccess && a128.numRegs == swa::kPPLaunchRegs &&
+                            a64.numRegs == swa::kPPLaunchRegs;
+        }
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::prefill_simt_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -285,6 +294,10 @@ int swa_forward(const void* q, const void* k, const void* v, void* out, int64_t 
         const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
         const char* impl = getenv("SWA_PREFILL_IMPL");
         if (!(impl && std::string(impl) == "tile")) {
+            if (!ds->pp_regs_ok)
+                return fail(SWA_ERR_UNSUPPORTED,
+                            "swa_forward: prefill kernel was not compiled with %d registers per thread",
+                            swa::kPPLaunchRegs);
             const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
             const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
             auto* ob = static_cast<__nv_bfloat16*>(out);
