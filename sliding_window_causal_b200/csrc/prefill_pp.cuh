@@ -112,13 +112,6 @@ __device__ __forceinline__ PPItem pp_decode(int u, int BH, int n_qt, int T, int 
     return it;
 }
 
-// Every lane of a role warp waits; the warp goes on only if all of them saw the phase.
-__device__ __forceinline__ bool pp_warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                             volatile int* abort) {
-    const bool ok = ptx::mbar_wait(bar, parity, limit_ns, abort);
-    return __all_sync(0xffffffffu, ok);
-}
-
 __device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W <= kPPPreciseWindow; }
 
 // Column of TMEM (relative to the S buffer) that holds P for keys 16kk..16kk+15: keys
@@ -301,9 +294,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     if (warp < 4) {
       ptx::regs_dec<kPPRoleRegs>();
       if (warp == 0) {
+        if (lane == 0) {
             // ------------------------------------------------------------ producer
-            // The whole warp runs the loop (warp-uniform values); lane 0 issues the copies.
-            const bool leader = lane == 0;
             bool ok = true;
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
@@ -312,43 +304,37 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (!ok || (x == 1 && !it.hasB)) break;
-                    if (nq[x] > 0) ok = pp_warp_wait(q_empty + x, (nq[x] - 1) & 1, wait_limit_ns, abort_flag);
+                    if (nq[x] > 0) ok = ptx::mbar_wait(q_empty + x, (nq[x] - 1) & 1, wait_limit_ns, abort_flag);
                     if (!ok) break;
-                    if (leader) {
-                        uint8_t* dst = smem + C::kQOff + x * C::kTileBytes;
-                        ptx::mbar_arrive_expect_tx(q_full + x, C::kTileBytes);
-                        for (int c = 0; c < D / 64; ++c)
-                            ptx::tma_load_3d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.bh);
-                    }
+                    uint8_t* dst = smem + C::kQOff + x * C::kTileBytes;
+                    ptx::mbar_arrive_expect_tx(q_full + x, C::kTileBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        ptx::tma_load_3d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.bh);
                     ++nq[x];
                 }
                 for (int kt = it.k0; kt <= it.k1 && ok; ++kt) {
                     for (int kv = 0; kv < 2; ++kv) {
                         const uint32_t st = loads % NS;
                         if (loads >= (uint32_t)NS)
-                            ok = pp_warp_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag);
+                            ok = ptx::mbar_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag);
                         if (!ok) break;
-                        if (leader) {
-                            uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
-                            ptx::mbar_arrive_expect_tx(ring_full + st, C::kTileBytes);
-                            for (int c = 0; c < D / 64; ++c)
-                                ptx::tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, ring_full + st, c * 64,
-                                                 kt * 128, it.bh);
-                        }
+                        uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
+                        ptx::mbar_arrive_expect_tx(ring_full + st, C::kTileBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            ptx::tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, ring_full + st, c * 64,
+                                             kt * 128, it.bh);
                         ++loads;
                     }
                 }
             }
-            if (!ok && leader) {
+            if (!ok) {
                 atomicCAS(status, 0, 5);
                 *abort_flag = 1;
             }
+        }
     } else if (warp == 1) {
-        {
+        if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
-            // The whole warp runs the loop so that descriptors and counters stay
-            // warp-uniform; lane 0 issues the MMAs and the commits.
-            const bool leader = lane == 0;
             // Descriptors: the high word (SBO = 1024, sm_100 version, 128-byte swizzle) is
             // the same for every operand; the low word is start >> 4 plus the leading byte
             // offset field, so each MMA needs one add (shared memory is far below 256 KiB, so
@@ -374,7 +360,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (x < nx && ok) ok = pp_warp_wait(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
+                    if (x < nx && ok) ok = ptx::mbar_wait(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
                 }
                 if (!ok) break;
                 int pend[2] = {-1, -1};
@@ -384,8 +370,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     const uint32_t j = (uint32_t)(kt - it.k0);
                     const uint32_t Lk = Lbase + 2 * j, Lv = Lk - 1;
                     const uint32_t stk = Lk % NS, stv = Lv % NS;
-                    if (kt <= it.k1) ok = pp_warp_wait(ring_full + stk, (Lk / NS) & 1, wait_limit_ns, abort_flag);
-                    if (ok && kt > it.k0) ok = pp_warp_wait(ring_full + stv, (Lv / NS) & 1, wait_limit_ns, abort_flag);
+                    if (kt <= it.k1) ok = ptx::mbar_wait(ring_full + stk, (Lk / NS) & 1, wait_limit_ns, abort_flag);
+                    if (ok && kt > it.k0) ok = ptx::mbar_wait(ring_full + stv, (Lv / NS) & 1, wait_limit_ns, abort_flag);
                     if (!ok) break;
                     const uint32_t k_lo = (ring_lo + stk * kStageLo) | lo_k;
                     const uint32_t v_lo = (ring_lo + stv * kStageLo) | lo_v;
@@ -394,57 +380,51 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                         if (x >= nx || !ok) break;
                         if (pend[x] >= 0) {
                             // PV_x(kt-1): needs P_x(kt-1), and O_x free if it starts the item
-                            ok = pp_warp_wait(p_full + x, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
+                            ok = ptx::mbar_wait(p_full + x, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
                             if (ok && first_pv[x] && ni[x] > 0)
-                                ok = pp_warp_wait(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
+                                ok = ptx::mbar_wait(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
                             if (!ok) break;
                             ptx::tc_fence_after();
-                            if (leader) {
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
+                                            desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
+                                            (!first_pv[x] || kk > 0) ? 1u : 0u);
+                            if (prec[x]) {
 #pragma unroll
                                 for (int kk = 0; kk < 8; ++kk)
-                                    ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
-                                                desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
-                                                (!first_pv[x] || kk > 0) ? 1u : 0u);
-                                if (prec[x]) {
-#pragma unroll
-                                    for (int kk = 0; kk < 8; ++kk)
-                                        ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
-                                                    desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u);
-                                }
-                                if (pend[x] == it.l[x]) ptx::tc_commit(o_final + x);
+                                    ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u);
                             }
                             first_pv[x] = false;
+                            if (pend[x] == it.l[x]) ptx::tc_commit(o_final + x);
                             pend[x] = -1;
                         } else {
                             ptx::tc_fence_after();
                         }
                         if (kt <= it.k1 && kt >= it.f[x] && kt <= it.l[x]) {
                             // S_x(kt) = Q_x K(kt)^T
-                            if (leader) {
 #pragma unroll
-                                for (int kk = 0; kk < D / 16; ++kk) {
-                                    const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                                    ptx::mma_ss(tmem + C::colS(x), desc_hi | (q_lo[x] + off), desc_hi | (k_lo + off),
-                                                idesc_s, kk > 0 ? 1u : 0u);
-                                }
-                                ptx::tc_commit(s_full + x);
-                                if (kt == it.l[x]) ptx::tc_commit(q_empty + x);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                                ptx::mma_ss(tmem + C::colS(x), desc_hi | (q_lo[x] + off), desc_hi | (k_lo + off),
+                                            idesc_s, kk > 0 ? 1u : 0u);
                             }
+                            ptx::tc_commit(s_full + x);
                             ++ns[x];
+                            if (kt == it.l[x]) ptx::tc_commit(q_empty + x);
                             pend[x] = kt;
                         }
                     }
                     if (!ok) break;
-                    if (leader) {
-                        if (kt <= it.k1) ptx::tc_commit(ring_empty + stk);  // K(kt) read by its S MMAs
-                        if (kt > it.k0) ptx::tc_commit(ring_empty + stv);   // V(kt-1) read by its PV MMAs
-                    }
+                    if (kt <= it.k1) ptx::tc_commit(ring_empty + stk);  // K(kt) read by its S MMAs
+                    if (kt > it.k0) ptx::tc_commit(ring_empty + stv);   // V(kt-1) read by its PV MMAs
                 }
                 L = Lbase + 2u * (uint32_t)(it.k1 - it.k0 + 1);
                 ++ni[0];
                 if (it.hasB) ++ni[1];
             }
-            if (!ok && leader) {
+            if (!ok) {
                 atomicCAS(status, 0, 5);
                 *abort_flag = 1;
             }

@@ -19,7 +19,6 @@
 #include "plan.h"
 #include "prefill_simt.cuh"
 #include "prefill_pp.cuh"
-#include "prefill_tc.cuh"
 
 // Per-device status word: kernels record the first error here (atomicCAS from 0).
 __device__ int g_swa_status = 0;
@@ -91,13 +90,7 @@ int device_state(DeviceState** out) {
         }
     }
     if (!st.attrs_set) {
-        e = cudaFuncSetAttribute(swa::prefill_tc_kernel<128, 3>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 swa::TcCfg<128, 3>::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(swa::prefill_tc_kernel<64, 4>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::TcCfg<64, 4>::kSmemBytes);
+        e = cudaSuccess;
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::prefill_pp_kernel<128>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -284,41 +277,27 @@ int swa_forward(const void* q, const void* k, const void* v, void* out, int64_t 
         if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
             return fail(SWA_ERR_MISALIGNED, "swa_forward: bf16 tensors must be 16-byte aligned");
         const int64_t BH = B * H;
-        const int n_qt = (int)((T + swa::kTileM - 1) / swa::kTileM);
+        const int n_qt = (int)((T + 127) / 128);
         if ((int64_t)n_qt * BH > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "swa_forward: too many tiles");
-        CUtensorMap mq, mk, mv, mo;
+        CUtensorMap mq, mk, mv;
         int rc;
         if ((rc = make_map(&mq, q, BH, T, D)) || (rc = make_map(&mk, k, BH, T, D)) ||
-            (rc = make_map(&mv, v, BH, T, D)) || (rc = make_map(&mo, out, BH, T, D)))
+            (rc = make_map(&mv, v, BH, T, D)))
             return rc;
         const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-        const char* impl = getenv("SWA_PREFILL_IMPL");
-        if (!(impl && std::string(impl) == "tile")) {
-            if (!ds->pp_regs_ok)
-                return fail(SWA_ERR_UNSUPPORTED,
-                            "swa_forward: prefill kernel was not compiled with %d registers per thread",
-                            swa::kPPLaunchRegs);
-            const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
-            const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
-            auto* ob = static_cast<__nv_bfloat16*>(out);
-            if (D == 128)
-                swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
-                    mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-            else
-                swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
-                    mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-            cudaError_t e = cudaGetLastError();
-            if (e != cudaSuccess) return cuda_fail(e, "swa_forward launch");
-            return success();
-        }
-        const dim3 grid((unsigned)(n_qt * BH));
-        if (D == 128) {
-            swa::prefill_tc_kernel<128, 3><<<grid, 192, swa::TcCfg<128, 3>::kSmemBytes, s>>>(
-                mq, mk, mv, mo, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-        } else {
-            swa::prefill_tc_kernel<64, 4><<<grid, 192, swa::TcCfg<64, 4>::kSmemBytes, s>>>(
-                mq, mk, mv, mo, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-        }
+        if (!ds->pp_regs_ok)
+            return fail(SWA_ERR_UNSUPPORTED,
+                        "swa_forward: prefill kernel was not compiled with %d registers per thread",
+                        swa::kPPLaunchRegs);
+        const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
+        const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
+        auto* ob = static_cast<__nv_bfloat16*>(out);
+        if (D == 128)
+            swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
+        else
+            swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
     } else {
         if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "swa_forward: fp32 supports D <= 4096");
         if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))

@@ -206,13 +206,18 @@ def test_window_sweep_sampled(wl):
 def test_growing_scores_move_the_reference(D, W):
     """Scores that grow steadily along the sequence (q . k_j grows with j) push every
     row's running maximum up by far more than the lazy-rescale threshold, tile after
-    tile and chunk after chunk inside a tile; the output must still match."""
+    tile; the output must still match.
+
+    Here a handful of keys dominate every row, so |out| is close to a single |v|. v is
+    drawn at half scale to keep |out| below about 1.5: at |out| >= 2 the bf16 output
+    spacing alone (0.0156) leaves half the 1e-2 budget to the bf16 weights P, which is
+    a property of bf16 outputs and bf16 P, not of the rescale path tested here."""
     T = 1500
     gen = torch.Generator().manual_seed(71)
     q = torch.ones(1, 2, T, D)
     k = (torch.arange(T, dtype=torch.float32) * 0.05)[None, None, :, None].expand(1, 2, T, D).clone()
     k += 0.01 * torch.randn(1, 2, T, D, generator=gen)
-    v = torch.randn(1, 2, T, D, generator=gen)
+    v = 0.5 * torch.randn(1, 2, T, D, generator=gen)
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
     out = run(q, k, v, W)
     ref = oracle.forward(f64(q), f64(k), f64(v), W)
