@@ -88,7 +88,9 @@ int swa_forward(const void* q, const void* k, const void* v, void* out,
  *   pos          : [B] int64, on the device, each >= 0.
  *   D            : 64 or 128. All pointers 16-byte aligned (pos 8-byte aligned).
  * The work is split along the ring into chunks whose partial softmax states are merged
- * in a fixed order (deterministic). The partial states live in a workspace that the
+ * in a fixed order (deterministic). The chunk length follows from the sizes (about 16
+ * CTAs per SM in total); the SWA_DECODE_CHUNK environment variable overrides it (in
+ * slots) for tuning. The partial states live in a workspace that the
  * library allocates with cudaMalloc on the first call for each (device, stream) and
  * keeps, growing it when a larger call needs more: make that first call before any
  * stream capture. Calls on one stream share its workspace; calls on different
@@ -110,6 +112,32 @@ int swa_device_status(void* stream);
 /* swa_last_error: message for the calling thread's last non-OK return ("" if none).
  * The pointer stays valid until the thread's next call into the library. */
 const char* swa_last_error(void);
+
+/*
+ * swa_decode_noalloc: swa_decode without any device allocation by the library.
+ *
+ * The source pages describe no counterpart of this entry point; it exists for callers
+ * that cannot let a library call cudaMalloc. Their device memory is owned end to end by
+ * another allocator (a framework's caching allocator, or a serving runtime that carves a
+ * fixed arena at start-up and counts any other allocation as a leak), or they run a
+ * latency-bound decode step that must not take the implicit device-wide synchronisation
+ * of cudaMalloc. Arguments, layout, results and errors are those of swa_decode, except:
+ *  - The split partial states and ticket counters live in one file-scope device array
+ *    of 4 MiB, which every GPU that loads the library holds until the process exits. The
+ *    library's own split plan (about 16 CTAs per SM) needs at most 2.5 MB for any size;
+ *    a request that would need more (B*H streams x splits x (D+2) floats plus B*H
+ *    counters, possible only when the SWA_DECODE_CHUNK environment variable forces a
+ *    small chunk) returns SWA_ERR_UNSUPPORTED with the byte count in swa_last_error()
+ *    and enqueues nothing; use swa_decode for it.
+ *  - The first call on a device looks up the array's device address and sets kernel
+ *    attributes (no allocation); make that first call before any stream capture.
+ *  - Every call shares the array and clears the counters it needs (cudaMemsetAsync on
+ *    `stream`). Calls whose kernels overlap on the GPU race on the array: keep them on one
+ *    stream, or otherwise ordered.
+ * The caller still owns and passes every input and output buffer.
+ */
+int swa_decode_noalloc(const void* q, const void* kring, const void* vring, const int64_t* pos,
+                       void* out, int64_t B, int64_t H, int64_t D, int64_t W, void* stream);
 
 /* ---- Host-side work planning (no GPU needed; the kernels use the same code) ---- */
 

@@ -10,7 +10,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_swa.so")
 
 # every exported symbol of include/swa.h
-EXPORTS = ("swa_forward", "swa_decode", "swa_device_status", "swa_last_error",
+EXPORTS = ("swa_forward", "swa_decode", "swa_decode_noalloc", "swa_device_status", "swa_last_error",
            "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
            "swa_set_wait_limit_ns", "swa_timeout_probe")
 
@@ -42,6 +42,8 @@ def lib(path=None):
     h.swa_forward.restype = i32
     h.swa_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     h.swa_decode.restype = i32
+    h.swa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    h.swa_decode_noalloc.restype = i32
     h.swa_device_status.argtypes = [vp]
     h.swa_device_status.restype = i32
     h.swa_last_error.argtypes = []

@@ -400,3 +400,96 @@ extern "C" int swa_timeout_probe(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "swa_timeout_probe launch");
     return success();
 }
+
+// ------------------------------------------------------------------ allocation-free decode
+// Some callers cannot let a library call cudaMalloc: their device memory is owned end to
+// end by another allocator (a framework's caching allocator, or a serving runtime that
+// carves a fixed arena at start-up and treats any other allocation as a leak), or they
+// run a latency-bound decode step that must not take cudaMalloc's implicit device-wide
+// synchronisation. For them, swa_decode_noalloc keeps the split partial states and ticket
+// counters in this fixed file-scope array instead of a cudaMalloc'd workspace. Every GPU
+// that loads the library holds the array until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+constexpr size_t kNoAllocCounterAlign = 256;
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[kNoAllocScratchBytes];
+
+std::map<int, void*> g_noalloc_scratch;  // device address of the array, per device
+
+// Once per device, with that device current: the array's name is only a host-side
+// stand-in in host code, so fetch the device address the kernels must be given.
+int noalloc_scratch(void** out) {
+    int dev;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_mu);
+    void*& ptr = g_noalloc_scratch[dev];
+    if (!ptr) {
+        e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+        if (e != cudaSuccess) {
+            ptr = nullptr;
+            return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+        }
+    }
+    *out = ptr;
+    return SWA_OK;
+}
+}  // namespace
+
+extern "C" int swa_decode_noalloc(const void* q, const void* kring, const void* vring,
+                                  const int64_t* pos, void* out, int64_t B, int64_t H, int64_t D,
+                                  int64_t W, void* stream) {
+    if (W < 1) return fail(SWA_ERR_INVALID_ARG, "swa_decode_noalloc: window W=%lld must be >= 1", (long long)W);
+    if (B < 0 || H < 0)
+        return fail(SWA_ERR_INVALID_ARG, "swa_decode_noalloc: negative size B=%lld H=%lld", (long long)B, (long long)H);
+    if (D < 1) return fail(SWA_ERR_INVALID_ARG, "swa_decode_noalloc: head dim D=%lld must be >= 1", (long long)D);
+    if (B == 0 || H == 0) return success();
+    if (!q || !kring || !vring || !pos || !out)
+        return fail(SWA_ERR_INVALID_ARG, "swa_decode_noalloc: null pointer");
+    if (D != 64 && D != 128)
+        return fail(SWA_ERR_UNSUPPORTED, "swa_decode_noalloc: D must be 64 or 128 (got %lld)", (long long)D);
+    if (!aligned(q, 16) || !aligned(kring, 16) || !aligned(vring, 16) || !aligned(out, 16) ||
+        !aligned(pos, 8))
+        return fail(SWA_ERR_MISALIGNED, "swa_decode_noalloc: tensors must be 16-byte aligned (pos 8-byte)");
+    if (B * H > INT32_MAX || W > INT32_MAX / 2 || B * H > INT64_MAX / W / D)
+        return fail(SWA_ERR_UNSUPPORTED, "swa_decode_noalloc: sizes too large");
+    int32_t S, chunk;
+    split_plan(B, H, D, W, &S, &chunk);
+    const size_t counter_bytes =
+        ((size_t)(B * H) * sizeof(int) + kNoAllocCounterAlign - 1) / kNoAllocCounterAlign * kNoAllocCounterAlign;
+    const size_t part_bytes = (size_t)(B * H) * S * (D + 2) * sizeof(float);
+    if (S > 1 && counter_bytes + part_bytes > kNoAllocScratchBytes)
+        return fail(SWA_ERR_UNSUPPORTED,
+                    "swa_decode_noalloc: %lld streams x %d splits need %zu bytes of scratch; the fixed "
+                    "array holds %zu (use swa_decode)",
+                    (long long)(B * H), (int)S, counter_bytes + part_bytes, kNoAllocScratchBytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    float* part = nullptr;
+    int* counters = nullptr;
+    if (S > 1) {
+        void* base;
+        if (int rc = noalloc_scratch(&base)) return rc;
+        counters = static_cast<int*>(base);
+        part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + counter_bytes);
+        // the array keeps the last call's contents: the ticket counters must start at zero
+        cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)(B * H) * sizeof(int), s);
+        if (e != cudaSuccess) return cuda_fail(e, "swa_decode_noalloc: clearing counters");
+    }
+    const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    const dim3 grid((unsigned)(B * H), (unsigned)S);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(kring);
+    const auto* vb = static_cast<const __nv_bfloat16*>(vring);
+    auto* ob = static_cast<__nv_bfloat16*>(out);
+    if (D == 128)
+        swa::decode_kernel<128><<<grid, swa::kDecodeWarps * 32, 0, s>>>(
+            qb, kb, vb, pos, ob, (int)H, (int)W, chunk, S, scale_log2, part, counters, ds->status);
+    else
+        swa::decode_kernel<64><<<grid, swa::kDecodeWarps * 32, 0, s>>>(
+            qb, kb, vb, pos, ob, (int)H, (int)W, chunk, S, scale_log2, part, counters, ds->status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swa_decode_noalloc launch");
+    return success();
+}

@@ -1,0 +1,70 @@
+"""The allocation-free decode entry point against the allocating one.
+
+swa_decode_noalloc serves callers that cannot let a library call cudaMalloc (device
+memory owned end to end by another allocator, or a latency-bound decode step that must
+not take cudaMalloc's device-wide synchronisation): it keeps its split partial states in
+a fixed 4 MiB array compiled into the library instead of a cudaMalloc'd workspace. Its
+results must match swa_decode, call after call, since every call shares that array.
+This file is collected last, so that a run which stops at the first failure has already
+run every other test; it also passes on its own in a fresh process.
+"""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import sliding_window_causal_b200 as swa
+from sliding_window_causal_b200 import _native, inputs
+from gpu_util import TOL
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def noalloc(q, kr, vr, pos, W, out):
+    B, H, D = q.shape
+    rc = _native.lib().swa_decode_noalloc(
+        q.data_ptr(), kr.data_ptr(), vr.data_ptr(), pos.data_ptr(), out.data_ptr(), B, H, D, W,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return rc
+
+
+CASES = [
+    # B, H, D, W, positions drawn from [0, pos_max)
+    (4, 2, 128, 300, 2000),     # many splits per stream
+    (3, 5, 64, 77, 500),
+    (16, 8, 128, 4096, 100000),  # two splits per stream
+    (64, 40, 64, 256, 1000),    # enough streams for a single split (no scratch)
+]
+
+
+@pytest.mark.parametrize("B,H,D,W,pos_max", CASES)
+def test_noalloc_matches_decode_on_consecutive_calls(B, H, D, W, pos_max):
+    q, kr, vr, pos = (t.to(DEV) for t in inputs.decode_inputs(B, H, D, W, pos_max, torch.bfloat16, 90 + W))
+    ref = swa.decode(q, kr, vr, pos, W)
+    swa.device_status()
+    tol = TOL[torch.bfloat16]
+    for _ in range(2):  # two calls in a row share the array
+        out = torch.full_like(q, float("nan"))
+        assert noalloc(q, kr, vr, pos, W, out) == 0, _native.lib().swa_last_error()
+        swa.device_status()
+        err = (out.float() - ref.float()).abs().max().item()
+        assert np.isfinite(err) and err <= tol, err
+
+
+def test_noalloc_rejects_requests_beyond_the_array(monkeypatch):
+    """A forced small chunk makes the partial states outgrow the fixed array: the call
+    is refused before anything is enqueued, with the sizes in the message."""
+    monkeypatch.setenv("SWA_DECODE_CHUNK", "32")
+    # 256 streams x 32 splits x 130 floats = 4.3 MB of partial states > 4 MiB. The buffers
+    # have their full sizes, so the call would be safe even if it were not refused.
+    B, H, D, W = 8, 32, 128, 1024
+    q = torch.zeros(B, H, D, dtype=torch.bfloat16, device=DEV)
+    r = torch.zeros(B, H, W, D, dtype=torch.bfloat16, device=DEV)
+    pos = torch.zeros(B, dtype=torch.int64, device=DEV)
+    out = torch.zeros_like(q)
+    assert noalloc(q, r, r, pos, W, out) == 2
+    assert b"scratch" in _native.lib().swa_last_error()
+    swa.device_status()
