@@ -32,8 +32,10 @@ def _load(path=None):
     lib.swa_oracle_forward_rows.argtypes = [d, d, d, i64, i64, i64, i64, i64, pi64, i64, d]
     lib.swa_oracle_weights.argtypes = [d, d, d, i64, i64, i64, i64, i64]
     lib.swa_oracle_decode.argtypes = [d, d, d, pi64, d, i64, i64, i64, i64]
+    lib.swa_oracle_forward_scaled.argtypes = [d, d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
+    lib.swa_oracle_weights_scaled.argtypes = [d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
     for f in (lib.swa_oracle_forward, lib.swa_oracle_forward_rows, lib.swa_oracle_weights,
-              lib.swa_oracle_decode):
+              lib.swa_oracle_decode, lib.swa_oracle_forward_scaled, lib.swa_oracle_weights_scaled):
         f.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -54,8 +56,9 @@ class OracleError(ValueError):
     pass
 
 
-def forward(q, k, v, W, lib=None):
-    """out[B,H,T,D] (float64) for q, k, v of shape [B,H,T,D] and window W."""
+def forward(q, k, v, W, lib=None, scale=None):
+    """out[B,H,T,D] (float64) for q, k, v of shape [B,H,T,D] and window W. scale=None is
+    the default 1/sqrt(D); a number multiplies the dot products instead."""
     lib = lib or _load()
     q, pq = _f64(q)
     k, pk = _f64(k)
@@ -65,7 +68,10 @@ def forward(q, k, v, W, lib=None):
     B, H, T, D = q.shape
     out = np.empty_like(q)
     _, po = _f64(out)
-    rc = lib.swa_oracle_forward(pq, pk, pv, po, B, H, T, D, int(W))
+    if scale is None:
+        rc = lib.swa_oracle_forward(pq, pk, pv, po, B, H, T, D, int(W))
+    else:
+        rc = lib.swa_oracle_forward_scaled(pq, pk, pv, po, B, H, T, D, int(W), float(scale))
     if rc != 0:
         raise OracleError(f"oracle forward rejected its arguments (rc={rc})")
     return out
@@ -87,15 +93,18 @@ def forward_rows(q, k, v, W, rows, lib=None):
     return out
 
 
-def weights(q, k, W, lib=None):
-    """Attention weights [B,H,T,T] of the definition (small inputs only)."""
+def weights(q, k, W, lib=None, scale=None):
+    """Attention weights [B,H,T,T] of the definition (small inputs only); scale as forward."""
     lib = lib or _load()
     q, pq = _f64(q)
     k, pk = _f64(k)
     B, H, T, D = q.shape
     w = np.empty((B, H, T, T), dtype=np.float64)
     _, pw = _f64(w)
-    rc = lib.swa_oracle_weights(pq, pk, pw, B, H, T, D, int(W))
+    if scale is None:
+        rc = lib.swa_oracle_weights(pq, pk, pw, B, H, T, D, int(W))
+    else:
+        rc = lib.swa_oracle_weights_scaled(pq, pk, pw, B, H, T, D, int(W), float(scale))
     if rc != 0:
         raise OracleError(f"oracle weights rejected its arguments (rc={rc})")
     return w

@@ -41,8 +41,14 @@
  * window). For stream b at absolute position P the query attends to positions
  * max(0, P-W+1) .. P, in ascending position order, read from slot p mod W.
  *
+ * Scale: the *_scaled entry points multiply the dot products by a caller-given
+ * factor instead of 1/sqrt(D) ("Mistral Architecture > Implementation: Sliding
+ * Window Attention", Step 2: an optional scale that defaults to 1/sqrt(head_dim)).
+ * The plain entry points are those with scale = 1/sqrt(D).
+ *
  * Return codes: 0 on success, 1 for an invalid argument (W < 1, a negative size,
- * a null pointer, a negative position). On error nothing is written.
+ * a null pointer, a negative position, a non-finite scale). On error nothing is
+ * written.
  */
 #include <math.h>
 #include <stdint.h>
@@ -55,10 +61,10 @@
 /* One query row of the prefill definition. qi: [D]. kh, vh: [T, D] for one (b,h).
  * out: [D]. scores: scratch of at least min(i+1, W) doubles. */
 static void oracle_row(const double* qi, const double* kh, const double* vh,
-                       int64_t i, int64_t D, int64_t W, double* scores, double* out) {
+                       int64_t i, int64_t D, int64_t W, double scale, double* scores,
+                       double* out) {
     int64_t lo = i - W + 1;
     if (lo < 0) lo = 0;
-    const double inv_sqrt_d = 1.0 / sqrt((double)D);
 
     /* scores over the band, j ascending */
     double m = -INFINITY;
@@ -66,7 +72,7 @@ static void oracle_row(const double* qi, const double* kh, const double* vh,
         const double* kj = kh + j * D;
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += qi[d] * kj[d];
-        double s = dot * inv_sqrt_d;
+        double s = dot * scale;
         scores[j - lo] = s;
         if (s > m) m = s;
     }
@@ -88,10 +94,11 @@ static int check_sizes(int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
     return ORACLE_OK;
 }
 
-/* Full prefill: out[B,H,T,D] for every row. */
-int swa_oracle_forward(const double* q, const double* k, const double* v, double* out,
-                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
-    if (check_sizes(B, H, T, D, W) != ORACLE_OK) return ORACLE_INVALID;
+/* Full prefill: out[B,H,T,D] for every row, scores scaled by `scale`. */
+int swa_oracle_forward_scaled(const double* q, const double* k, const double* v, double* out,
+                              int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                              double scale) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK || !isfinite(scale)) return ORACLE_INVALID;
     if (B * H * T == 0) return ORACLE_OK;
     if (!q || !k || !v || !out) return ORACLE_INVALID;
     const int64_t nrows = B * H * T;
@@ -109,12 +116,19 @@ int swa_oracle_forward(const double* q, const double* k, const double* v, double
                 const int64_t bh = r / T, i = r % T;
                 const double* kh = k + bh * T * D;
                 const double* vh = v + bh * T * D;
-                oracle_row(q + r * D, kh, vh, i, D, W, scores, out + r * D);
+                oracle_row(q + r * D, kh, vh, i, D, W, scale, scores, out + r * D);
             }
             free(scores);
         }
     }
     return bad ? ORACLE_INVALID : ORACLE_OK;
+}
+
+/* Full prefill with the default scale 1/sqrt(D). */
+int swa_oracle_forward(const double* q, const double* k, const double* v, double* out,
+                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (D < 1) return ORACLE_INVALID;
+    return swa_oracle_forward_scaled(q, k, v, out, B, H, T, D, W, 1.0 / sqrt((double)D));
 }
 
 /* Selected rows only: rows[n] holds flattened row indices r = (b*H + h)*T + i.
@@ -140,8 +154,8 @@ int swa_oracle_forward_rows(const double* q, const double* k, const double* v,
             for (int64_t t = 0; t < n; ++t) {
                 const int64_t r = rows[t];
                 const int64_t bh = r / T, i = r % T;
-                oracle_row(q + r * D, k + bh * T * D, v + bh * T * D, i, D, W, scores,
-                           out_rows + t * D);
+                oracle_row(q + r * D, k + bh * T * D, v + bh * T * D, i, D, W,
+                           1.0 / sqrt((double)D), scores, out_rows + t * D);
             }
             free(scores);
         }
@@ -150,13 +164,14 @@ int swa_oracle_forward_rows(const double* q, const double* k, const double* v,
 }
 
 /* Attention weights of the definition, for checking probabilities on small
- * inputs: weights[B,H,T,T], zero outside the band, e_j / sum e_j inside. */
-int swa_oracle_weights(const double* q, const double* k, double* weights,
-                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
-    if (check_sizes(B, H, T, D, W) != ORACLE_OK) return ORACLE_INVALID;
+ * inputs: weights[B,H,T,T], zero outside the band, e_j / sum e_j inside, with the
+ * scores scaled by `scale`. */
+int swa_oracle_weights_scaled(const double* q, const double* k, double* weights,
+                              int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                              double scale) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK || !isfinite(scale)) return ORACLE_INVALID;
     if (B * H * T == 0) return ORACLE_OK;
     if (!q || !k || !weights) return ORACLE_INVALID;
-    const double inv_sqrt_d = 1.0 / sqrt((double)D);
     for (int64_t bh = 0; bh < B * H; ++bh) {
         for (int64_t i = 0; i < T; ++i) {
             double* wrow = weights + (bh * T + i) * T;
@@ -169,7 +184,7 @@ int swa_oracle_weights(const double* q, const double* k, double* weights,
                 const double* kj = k + (bh * T + j) * D;
                 double dot = 0.0;
                 for (int64_t d = 0; d < D; ++d) dot += qi[d] * kj[d];
-                wrow[j] = dot * inv_sqrt_d;
+                wrow[j] = dot * scale;
                 if (wrow[j] > m) m = wrow[j];
             }
             double denom = 0.0;
@@ -181,6 +196,13 @@ int swa_oracle_weights(const double* q, const double* k, double* weights,
         }
     }
     return ORACLE_OK;
+}
+
+/* Attention weights with the default scale 1/sqrt(D). */
+int swa_oracle_weights(const double* q, const double* k, double* weights,
+                       int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (D < 1) return ORACLE_INVALID;
+    return swa_oracle_weights_scaled(q, k, weights, B, H, T, D, W, 1.0 / sqrt((double)D));
 }
 
 /* Decode over a rolling buffer. q: [B,H,D]; kring, vring: [B,H,W,D]; pos: [B];

@@ -20,11 +20,11 @@ from golden import read_band, read_moving_average
 TIGHT = 1e-12
 
 
-def _sdpa(q, k, v, mask=None, causal=False):
+def _sdpa(q, k, v, mask=None, causal=False, scale=None):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
     out = torch.nn.functional.scaled_dot_product_attention(
         t(q), t(k), t(v), attn_mask=None if mask is None else torch.from_numpy(mask),
-        dropout_p=0.0, is_causal=causal)
+        dropout_p=0.0, is_causal=causal, scale=scale)
     return out.numpy()
 
 
@@ -219,6 +219,50 @@ def pin_shapes(lib):
     assert out.shape == (1, 5, 3)
 
 
+def pin_scaled(lib):
+    """A caller-given scale ("Mistral Architecture > Implementation: Sliding Window
+    Attention", Step 2): torch's scaled dot-product attention with the same scale and the
+    brute-force band mask agrees; scale 0 gives the trailing mean of v whatever q and k
+    hold; scaling q by a and the scale by 1/a changes nothing; and the default scale is
+    1/sqrt(D)."""
+    rng = np.random.default_rng(41)
+    for (B, H, T, D, W) in ((1, 2, 9, 4, 3), (2, 1, 20, 8, 6), (1, 2, 14, 3, 20)):
+        q, k, v = (_rand(rng, B, H, T, D) for _ in range(3))
+        for sc in (0.05, 0.5, 1.0, 2.0, -0.7):
+            out = oracle.forward(q, k, v, W, lib=lib, scale=sc)
+            ref = _sdpa(q, k, v, mask=brute.band_mask(T, W), scale=sc)
+            assert np.abs(out - ref).max() <= TIGHT, f"sdpa scale={sc} T={T} W={W}"
+        out0 = oracle.forward(q, k, v, W, lib=lib, scale=0.0)
+        for i in range(T):
+            lo = max(0, i - W + 1)
+            assert np.abs(out0[:, :, i, :] - v[:, :, lo:i + 1, :].mean(axis=2)).max() <= TIGHT
+        a = 3.0
+        o1 = oracle.forward(q * a, k, v, W, lib=lib, scale=0.25 / a)
+        o2 = oracle.forward(q, k, v, W, lib=lib, scale=0.25)
+        assert np.abs(o1 - o2).max() <= TIGHT, "homogeneity in q and the scale"
+        d = oracle.forward(q, k, v, W, lib=lib, scale=1.0 / np.sqrt(D))
+        assert np.array_equal(d, oracle.forward(q, k, v, W, lib=lib)), "default scale"
+
+
+def pin_weights_scaled(lib):
+    """Weights with a caller-given scale equal torch's softmax of the scaled, band-masked
+    score matrix built with torch.matmul; scale 0 spreads each row evenly over its band."""
+    rng = np.random.default_rng(43)
+    B, H, T, D, W = 1, 2, 13, 5, 4
+    q, k = (_rand(rng, B, H, T, D) for _ in range(2))
+    mask = brute.band_mask(T, W)
+    for sc in (0.3, 1.7, -1.1):
+        w = oracle.weights(q, k, W, lib=lib, scale=sc)
+        sco = torch.matmul(torch.from_numpy(q), torch.from_numpy(k).transpose(-1, -2)) * sc
+        sco = sco.masked_fill(~torch.from_numpy(mask), float("-inf"))
+        ref = torch.softmax(sco, dim=-1).numpy()
+        assert np.abs(w - ref).max() <= TIGHT, f"weights scale={sc}"
+    w0 = oracle.weights(q, k, W, lib=lib, scale=0.0)
+    counts = np.minimum(np.arange(T) + 1, W)
+    even = np.where(mask, 1.0 / counts[:, None], 0.0)
+    assert np.abs(w0 - even).max() <= TIGHT, "scale 0 gives even weights"
+
+
 ALL_PINS = [pin_band_masks, pin_moving_average, pin_trailing_mean_any_k, pin_causal_reduction,
             pin_general_band, pin_window_one, pin_independence, pin_weights, pin_rows_subset,
-            pin_decode, pin_shapes]
+            pin_decode, pin_shapes, pin_scaled, pin_weights_scaled]

@@ -29,7 +29,10 @@ MUTANTS = [
      [("int64_t lo = i - W + 1;", "int64_t lo = i - W;")] + WIDER_SCRATCH),
     ("band one key narrower", [("int64_t lo = i - W + 1;", "int64_t lo = i - W + 2;")]),
     ("scale 1/D instead of 1/sqrt(D)", [("1.0 / sqrt((double)D)", "1.0 / (double)D")]),
-    ("no scale", [("double s = dot * inv_sqrt_d;", "double s = dot;")]),
+    ("prefill ignores the scale", [("double s = dot * scale;", "double s = dot;")]),
+    ("decode ignores the scale", [("double s = dot * inv_sqrt_d;", "double s = dot;")]),
+    ("weights ignore the scale", [("wrow[j] = dot * scale;", "wrow[j] = dot;")]),
+    ("scale applied twice", [("double s = dot * scale;", "double s = dot * scale * scale;")]),
     ("scores read v instead of k",
      [("const double* kj = kh + j * D;", "const double* kj = vh + j * D;")]),
     ("exponent sign flipped", [("exp(scores[j - lo] - m)", "exp(m - scores[j - lo])")]),
