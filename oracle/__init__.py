@@ -34,8 +34,11 @@ def _load(path=None):
     lib.swa_oracle_decode.argtypes = [d, d, d, pi64, d, i64, i64, i64, i64]
     lib.swa_oracle_forward_scaled.argtypes = [d, d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
     lib.swa_oracle_weights_scaled.argtypes = [d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
+    lib.swa_oracle_chunk.argtypes = [d, d, d, d, d, pi64, d, i64, i64, i64, i64, i64]
+    lib.swa_oracle_ring_append.argtypes = [d, d, d, d, pi64, i64, i64, i64, i64, i64]
     for f in (lib.swa_oracle_forward, lib.swa_oracle_forward_rows, lib.swa_oracle_weights,
-              lib.swa_oracle_decode, lib.swa_oracle_forward_scaled, lib.swa_oracle_weights_scaled):
+              lib.swa_oracle_decode, lib.swa_oracle_forward_scaled, lib.swa_oracle_weights_scaled,
+              lib.swa_oracle_chunk, lib.swa_oracle_ring_append):
         f.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -126,6 +129,48 @@ def decode(q, kring, vring, pos, W, lib=None):
     if rc != 0:
         raise OracleError(f"oracle decode rejected its arguments (rc={rc})")
     return out
+
+
+def chunk(q, kc, vc, kring, vring, pos, W, lib=None):
+    """out[B,H,C,D] for a chunk of C new tokens per stream (positions pos[b] ..
+    pos[b]+C-1) over the rolling buffer that holds the positions before it."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    kc, pkc = _f64(kc)
+    vc, pvc = _f64(vc)
+    kring, pkr = _f64(kring)
+    vring, pvr = _f64(vring)
+    pos, pp = _i64(pos)
+    B, H, C, D = q.shape
+    if kc.shape != q.shape or vc.shape != q.shape or kring.shape != (B, H, W, D) or \
+            vring.shape != (B, H, W, D) or pos.shape != (B,):
+        raise OracleError("chunk: q/k/v [B,H,C,D], rings [B,H,W,D], pos [B]")
+    out = np.empty_like(q)
+    _, po = _f64(out)
+    rc = lib.swa_oracle_chunk(pq, pkc, pvc, pkr, pvr, pp, po, B, H, C, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle chunk rejected its arguments (rc={rc})")
+    return out
+
+
+def ring_append(kc, vc, kring, vring, pos, W, lib=None):
+    """New (kring, vring) after the chunk's positions pos[b] .. pos[b]+C-1 enter the
+    ring, position p into slot p mod W (the inputs are not modified)."""
+    lib = lib or _load()
+    kc, pkc = _f64(kc)
+    vc, pvc = _f64(vc)
+    kring = np.array(kring, dtype=np.float64, copy=True, order="C")
+    vring = np.array(vring, dtype=np.float64, copy=True, order="C")
+    pkr = kring.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    pvr = vring.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    pos, pp = _i64(pos)
+    B, H, C, D = kc.shape
+    if vc.shape != kc.shape or kring.shape != (B, H, W, D) or vring.shape != (B, H, W, D):
+        raise OracleError("ring_append: k/v [B,H,C,D], rings [B,H,W,D]")
+    rc = lib.swa_oracle_ring_append(pkc, pvc, pkr, pvr, pp, B, H, C, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle ring_append rejected its arguments (rc={rc})")
+    return kring, vring
 
 
 def load_variant(path):

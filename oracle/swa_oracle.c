@@ -260,3 +260,93 @@ int swa_oracle_decode(const double* q, const double* kring, const double* vring,
     }
     return bad ? ORACLE_INVALID : ORACLE_OK;
 }
+
+/* Chunked streaming prefill. Stream b has seen positions 0 .. pos[b]-1; the ring
+ * holds the last min(pos[b], W) of them, position p in slot p mod W
+ * ("25. Sliding-Window Causal Attention for Streaming Inference", Problem: a bounded
+ * KV cache that keeps only the window; "Sliding Window Attention", Advantages: a KV
+ * cache of size W). A chunk of C new tokens takes positions pos[b] .. pos[b]+C-1:
+ * q, kc, vc, out are [B,H,C,D], kring, vring [B,H,W,D]. Query c, at position
+ * P = pos[b] + c, attends to positions max(0, P-W+1) .. P in ascending order, with
+ * the same formula as a prefill row: a position p < pos[b] is read from ring slot
+ * p mod W, a position p >= pos[b] from chunk row p - pos[b]. */
+static void oracle_chunk_one(const double* qc, const double* kcs, const double* vcs,
+                             const double* kr, const double* vr, int64_t pos0, int64_t c,
+                             int64_t D, int64_t W, double* scores, double* out) {
+    const int64_t P = pos0 + c;
+    int64_t first = P - W + 1;
+    if (first < 0) first = 0;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double m = -INFINITY;
+    for (int64_t p = first; p <= P; ++p) {
+        const double* kp = (p < pos0) ? kr + (p % W) * D : kcs + (p - pos0) * D;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qc[d] * kp[d];
+        double s = dot * inv_sqrt_d;
+        scores[p - first] = s;
+        if (s > m) m = s;
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    double denom = 0.0;
+    for (int64_t p = first; p <= P; ++p) {
+        double e = exp(scores[p - first] - m);
+        denom += e;
+        const double* vp = (p < pos0) ? vr + (p % W) * D : vcs + (p - pos0) * D;
+        for (int64_t d = 0; d < D; ++d) out[d] += e * vp[d];
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] = out[d] / denom;
+}
+
+int swa_oracle_chunk(const double* q, const double* kc, const double* vc,
+                     const double* kring, const double* vring, const int64_t* pos,
+                     double* out, int64_t B, int64_t H, int64_t C, int64_t D, int64_t W) {
+    if (W < 1 || B < 0 || H < 0 || C < 0 || D < 1) return ORACLE_INVALID;
+    if (B * H * C == 0) return ORACLE_OK;
+    if (!q || !kc || !vc || !kring || !vring || !pos || !out) return ORACLE_INVALID;
+    for (int64_t b = 0; b < B; ++b)
+        if (pos[b] < 0) return ORACLE_INVALID;
+    const int64_t nrows = B * H * C;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* scores = (double*)malloc((size_t)W * sizeof(double));
+        if (!scores) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t r = 0; r < nrows; ++r) {
+                const int64_t bh = r / C, c = r % C, b = bh / H;
+                oracle_chunk_one(q + r * D, kc + bh * C * D, vc + bh * C * D,
+                                 kring + bh * W * D, vring + bh * W * D, pos[b], c, D, W,
+                                 scores, out + r * D);
+            }
+            free(scores);
+        }
+    }
+    return bad ? ORACLE_INVALID : ORACLE_OK;
+}
+
+/* Ring append: the chunk's positions pos[b] .. pos[b]+C-1 enter the ring in order,
+ * position p into slot p mod W, each overwriting what the slot held. kc, vc:
+ * [B,H,C,D]; kring, vring: [B,H,W,D], updated in place. */
+int swa_oracle_ring_append(const double* kc, const double* vc, double* kring, double* vring,
+                           const int64_t* pos, int64_t B, int64_t H, int64_t C, int64_t D,
+                           int64_t W) {
+    if (W < 1 || B < 0 || H < 0 || C < 0 || D < 1) return ORACLE_INVALID;
+    if (B * H * C == 0) return ORACLE_OK;
+    if (!kc || !vc || !kring || !vring || !pos) return ORACLE_INVALID;
+    for (int64_t b = 0; b < B; ++b)
+        if (pos[b] < 0) return ORACLE_INVALID;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H;
+        for (int64_t c = 0; c < C; ++c) {
+            const int64_t slot = (pos[b] + c) % W;
+            for (int64_t d = 0; d < D; ++d) {
+                kring[(bh * W + slot) * D + d] = kc[(bh * C + c) * D + d];
+                vring[(bh * W + slot) * D + d] = vc[(bh * C + c) * D + d];
+            }
+        }
+    }
+    return ORACLE_OK;
+}

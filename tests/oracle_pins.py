@@ -263,6 +263,60 @@ def pin_weights_scaled(lib):
     assert np.abs(w0 - even).max() <= TIGHT, "scale 0 gives even weights"
 
 
+def pin_chunk_stream(lib):
+    """A stream fed chunk by chunk: each chunk's outputs over the ring (built position by
+    position from the history) equal the same rows of torch's scaled dot-product
+    attention over the whole history with the brute-force band mask; a chunk of one
+    token equals decode."""
+    rng = np.random.default_rng(47)
+    D, H, B = 4, 2, 1
+    for W in (1, 3, 8):
+        for (pos0, C) in ((0, 5), (0, 1), (2, 4), (W - 1, 3), (W, 1), (W + 2, 2 * W + 1),
+                          (3 * W + 1, W), (5, 12)):
+            T = pos0 + C
+            qh, kh, vh = (_rand(rng, B, H, T, D) for _ in range(3))
+            ref = _sdpa(qh, kh, vh, mask=brute.band_mask(T, W))[:, :, pos0:, :]
+            kr = np.zeros((B, H, W, D))
+            vr = np.zeros((B, H, W, D))
+            if pos0 > 0:
+                for h in range(H):
+                    kr[0, h], vr[0, h] = _ring_from_history(kh[0, h], vh[0, h], pos0 - 1, W)
+            pos = np.array([pos0])
+            out = oracle.chunk(qh[:, :, pos0:], kh[:, :, pos0:], vh[:, :, pos0:], kr, vr, pos, W,
+                               lib=lib)
+            assert np.abs(out - ref).max() <= TIGHT, f"chunk W={W} pos={pos0} C={C}"
+            if C == 1:
+                kr2, vr2 = kr.copy(), vr.copy()
+                kr2[:, :, pos0 % W], vr2[:, :, pos0 % W] = kh[:, :, pos0], vh[:, :, pos0]
+                dec = oracle.decode(qh[:, :, pos0], kr2, vr2, pos, W, lib=lib)
+                assert np.abs(out[:, :, 0] - dec).max() <= TIGHT, "one-token chunk is decode"
+
+
+def pin_ring_append(lib):
+    """Appending a history in chunks of any sizes leaves the ring that writing it
+    position by position leaves (brute force), whatever the chunking."""
+    rng = np.random.default_rng(53)
+    D, H = 3, 2
+    for W in (1, 4, 7):
+        T = 3 * W + 5
+        kh, vh = _rand(rng, 1, H, T, D), _rand(rng, 1, H, T, D)
+        for sizes in ([T], [1] * T, [W + 2, 1, T - W - 3], [2, W, W, T - 2 - 2 * W]):
+            kr = np.full((1, H, W, D), np.nan)
+            vr = np.full((1, H, W, D), np.nan)
+            p = 0
+            for c in sizes:
+                kr, vr = oracle.ring_append(kh[:, :, p:p + c], vh[:, :, p:p + c], kr, vr,
+                                            np.array([p]), W, lib=lib)
+                p += c
+                for h in range(H):
+                    ek, ev = _ring_from_history(kh[0, h], vh[0, h], p - 1, W)
+                    n = min(p, W)
+                    slots = [q % W for q in range(p - n, p)]
+                    assert np.array_equal(kr[0, h, slots], ek[slots]), f"ring k W={W} {sizes}"
+                    assert np.array_equal(vr[0, h, slots], ev[slots]), f"ring v W={W} {sizes}"
+
+
 ALL_PINS = [pin_band_masks, pin_moving_average, pin_trailing_mean_any_k, pin_causal_reduction,
             pin_general_band, pin_window_one, pin_independence, pin_weights, pin_rows_subset,
-            pin_decode, pin_shapes, pin_scaled, pin_weights_scaled]
+            pin_decode, pin_shapes, pin_scaled, pin_weights_scaled, pin_chunk_stream,
+            pin_ring_append]

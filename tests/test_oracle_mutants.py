@@ -42,6 +42,12 @@ MUTANTS = [
     ("decode wrong slot", [("(p % W) * D", "((p + 1) % W) * D")]),
     ("decode one extra position",
      [("int64_t first = P - W + 1;", "int64_t first = P - W;")] + WIDER_SCRATCH),
+    ("chunk reads its own first position from the ring",
+     [("(p < pos0) ? kr + (p % W) * D", "(p <= pos0) ? kr + (p % W) * D")]),
+    ("chunk band one key wider",
+     [("int64_t first = P - W + 1;\n    if (first < 0) first = 0;\n    const double inv_sqrt_d = 1.0 / sqrt((double)D);\n    double m = -INFINITY;\n    for (int64_t p = first; p <= P; ++p) {\n        const double* kp = (p < pos0)",
+       "int64_t first = P - W;\n    if (first < 0) first = 0;\n    const double inv_sqrt_d = 1.0 / sqrt((double)D);\n    double m = -INFINITY;\n    for (int64_t p = first; p <= P; ++p) {\n        const double* kp = (p < pos0)")] + WIDER_SCRATCH),
+    ("ring append one slot late", [("(pos[b] + c) % W", "(pos[b] + c + 1) % W")]),
     ("weights unnormalised", [("wrow[j] = wrow[j] / denom;", "wrow[j] = wrow[j];")]),
 ]
 
