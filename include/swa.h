@@ -18,8 +18,9 @@
  * used; a caller who wants it passes W+1.
  *
  * Conventions for every call below:
- *  - Every tensor pointer is a DEVICE pointer to row-major contiguous memory, owned
- *    by the caller. The library keeps no pointer after a call returns.
+ *  - Every tensor pointer is a DEVICE pointer to row-major contiguous memory (or to a
+ *    strided view, where a call takes strides), owned by the caller. The library keeps
+ *    no pointer after a call returns.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *    Calls enqueue work on it and return without waiting (asynchronous).
  *  - Calls return an swa_status code and never throw. All validation happens before
@@ -71,6 +72,51 @@ typedef enum {
 int swa_forward(const void* q, const void* k, const void* v, void* out,
                 int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
                 int dtype, void* stream);
+
+/*
+ * swa_forward_ex: swa_forward with a caller-chosen score scale and strided operands.
+ *
+ * "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2) takes its
+ * inputs as (batch, seq_len, num_heads, head_dim) and an optional scale that defaults to
+ * 1/sqrt(head_dim). This call covers both:
+ *   scale   : scores are (q . k) * scale. swa_forward is scale = 1/sqrt(D). SWA_BF16 takes
+ *             any scale > 0 (the tensor-core softmax scales the row maximum of the raw
+ *             scores, which is the maximum of the scaled ones only for a positive scale);
+ *             SWA_F32 takes any finite value, 0 giving equal weights over the band (a
+ *             trailing moving average of v).
+ *   strides : NULL for contiguous [B,H,T,D], or 12 element strides (not bytes), in the
+ *             order q(b,h,t), k(b,h,t), v(b,h,t), out(b,h,t); the head dimension is always
+ *             contiguous. Element (b,h,t,d) of q is at q + b*s[0] + h*s[1] + t*s[2] + d.
+ *             The [B,T,H,D] layout of the page is (T*H*D, D, H*D) for every operand.
+ *             The stride of a size-1 dimension is ignored. The rows of out must not overlap
+ *             each other or the inputs; this is documented, not checked.
+ * Everything else is as swa_forward. Extra errors: a non-finite scale, or a negative
+ * stride or one above 2^38 -> SWA_ERR_INVALID_ARG; for SWA_BF16 a scale <= 0 ->
+ * SWA_ERR_UNSUPPORTED, and a stride that is not a multiple of 8 elements (16 bytes) ->
+ * SWA_ERR_MISALIGNED.
+ */
+int swa_forward_ex(const void* q, const void* k, const void* v, void* out,
+                   int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                   double scale, const int64_t* strides, int dtype, void* stream);
+
+/*
+ * swa_band_weights: the softmax weights of every query's band, for inspection.
+ *
+ * "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2) returns the
+ * attention weights beside the output. Outside the band they are zero, so only the band is
+ * written: weights is [B, H, T, Wo] fp32 contiguous with Wo = min(W, T), and
+ * weights[b,h,i,c] is the weight of key j = i - Wo + 1 + c (c = Wo-1 is the query itself),
+ * or 0 where j < 0. Each row of weights sums to 1 (up to fp32 rounding). The weights are
+ * computed in fp32 on the CUDA cores, from q and k of `dtype` (SWA_F32 or SWA_BF16).
+ *   q, k    : [B,H,T,D] device tensors; strides NULL (contiguous) or 6 element strides
+ *             q(b,h,t), k(b,h,t) as in swa_forward_ex. D <= 4096.
+ *   scale   : as swa_forward_ex (pass 1/sqrt(D) for the scores of swa_forward).
+ * This is a debugging aid: it writes B*H*T*Wo*4 bytes, so it is not on the prefill path.
+ * Errors: as swa_forward_ex; pointers must be aligned to their element size.
+ */
+int swa_band_weights(const void* q, const void* k, float* weights,
+                     int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                     double scale, const int64_t* strides, int dtype, void* stream);
 
 /*
  * swa_decode: one new query per stream against a W-slot rolling KV buffer.

@@ -5,7 +5,10 @@ does all the work; these functions check torch tensors, pass their device pointe
 and the current CUDA stream to the C ABI, and raise SwaError on a non-OK status.
 PyTorch only supplies device memory and streams.
 
-    forward(q, k, v, window)            prefill, q/k/v [B,H,T,D] bf16 (D 64|128) or fp32
+    forward(q, k, v, window, scale=None)  prefill, q/k/v [B,H,T,D] views (bf16 D 64|128, or
+                                        fp32), any (b,h,t) strides, e.g. q.transpose(1, 2)
+                                        of a [B,T,H,D] tensor
+    band_weights(q, k, window)          the softmax weights of each band, [B,H,T,min(W,T)]
     decode(q, kring, vring, pos, window)  one query per stream over a W-slot ring
     forward_host(...)                   prefill from pinned host tensors (copies included)
 """
@@ -14,7 +17,7 @@ import ctypes
 from . import _native
 from ._native import SWA_BF16, SWA_F32, SwaError, check
 
-__all__ = ["forward", "decode", "forward_host", "device_status", "tile_class", "valid_slots",
+__all__ = ["forward", "band_weights", "decode", "forward_host", "device_status", "tile_class", "valid_slots",
            "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
 
 
@@ -37,22 +40,32 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
 
 
-def _need_cuda(*ts):
+def _need_cuda(*ts, contiguous=True):
     for t in ts:
         if not t.is_cuda:
             raise ValueError("tensors must be on a CUDA device (use forward_host for host tensors)")
-        if not t.is_contiguous():
+        if contiguous and not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if not contiguous and t.dim() > 0 and t.shape[-1] > 1 and t.stride(-1) != 1:
+            raise ValueError("the head dimension must be contiguous (stride 1)")
     dev = ts[0].device
     if any(t.device != dev for t in ts):
         raise ValueError("tensors must be on one device")
     return dev
 
 
-def forward(q, k, v, window, out=None):
-    """Sliding-window causal attention prefill. q, k, v: [B,H,T,D] contiguous CUDA
-    tensors of one dtype (bf16 with D in {64, 128}, or fp32 with any D <= 4096).
-    A 3-D [B,T,D] input is treated as one head. Returns out (same shape and dtype)."""
+def _bht_strides(*ts):
+    """(b, h, t) element strides of [B,H,T,D] views, flattened, as a ctypes int64 array."""
+    vals = [x for t in ts for x in t.stride()[:3]]
+    return (ctypes.c_int64 * len(vals))(*vals)
+
+
+def forward(q, k, v, window, out=None, scale=None):
+    """Sliding-window causal attention prefill. q, k, v: [B,H,T,D] CUDA tensors of one
+    dtype (bf16 with D in {64, 128}, or fp32 with any D <= 4096), each with a contiguous
+    head dimension and any (b,h,t) strides: a [B,T,H,D] tensor is passed as
+    x.transpose(1, 2). A 3-D [B,T,D] input is treated as one head. scale defaults to
+    1/sqrt(D). Returns out (same shape and dtype; allocated with q's strides if None)."""
     torch = _torch()
     squeeze = q.dim() == 3
     if squeeze:
@@ -63,18 +76,46 @@ def forward(q, k, v, window, out=None):
         raise ValueError("q, k, v must share one [B,H,T,D] shape")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
-    dev = _need_cuda(q, k, v)
+    dev = _need_cuda(q, k, v, contiguous=False)
     if out is None:
         out = torch.empty_like(q)
     else:
-        _need_cuda(out)
+        _need_cuda(out, contiguous=False)
         if out.shape != q.shape or out.dtype != q.dtype:
             raise ValueError("out must match q")
     B, H, T, D = q.shape
+    lib = _native.lib()
     with torch.cuda.device(dev):
-        check(_native.lib().swa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                        B, H, T, D, int(window), _dtype_code(q), _stream_ptr(dev)))
+        if scale is None and all(t.is_contiguous() for t in (q, k, v, out)):
+            check(lib.swa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  B, H, T, D, int(window), _dtype_code(q), _stream_ptr(dev)))
+        else:
+            sc = 1.0 / D ** 0.5 if scale is None else float(scale)
+            check(lib.swa_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     B, H, T, D, int(window), sc, _bht_strides(q, k, v, out),
+                                     _dtype_code(q), _stream_ptr(dev)))
     return out.squeeze(1) if squeeze else out
+
+
+def band_weights(q, k, window, scale=None):
+    """Softmax weights of every query's band: a [B,H,T,Wo] fp32 tensor, Wo = min(W, T),
+    where [..., i, c] is the weight of key j = i - Wo + 1 + c (0 where j < 0). q, k as in
+    forward (bf16 or fp32, strided views allowed). A debugging aid, not the prefill path."""
+    torch = _torch()
+    if q.dim() != 4 or k.shape != q.shape:
+        raise ValueError("q and k must share one [B,H,T,D] shape")
+    if k.dtype != q.dtype:
+        raise TypeError("q and k must share one dtype")
+    dev = _need_cuda(q, k, contiguous=False)
+    B, H, T, D = q.shape
+    Wo = min(int(window), T) if window >= 1 else int(window)
+    w = torch.empty((B, H, T, max(Wo, 0)), dtype=torch.float32, device=dev)
+    sc = 1.0 / D ** 0.5 if scale is None else float(scale)
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_band_weights(q.data_ptr(), k.data_ptr(), w.data_ptr(), B, H, T, D,
+                                             int(window), sc, _bht_strides(q, k), _dtype_code(q),
+                                             _stream_ptr(dev)))
+    return w
 
 
 def decode(q, kring, vring, pos, window, out=None):

@@ -10,8 +10,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_swa.so")
 
 # every exported symbol of include/swa.h
-EXPORTS = ("swa_forward", "swa_decode", "swa_decode_noalloc", "swa_device_status", "swa_last_error",
-           "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
+EXPORTS = ("swa_forward", "swa_forward_ex", "swa_band_weights", "swa_decode", "swa_decode_noalloc",
+           "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
            "swa_set_wait_limit_ns", "swa_timeout_probe")
 
 SWA_F32, SWA_BF16 = 0, 1
@@ -40,6 +40,12 @@ def lib(path=None):
     i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
     h.swa_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, vp]
     h.swa_forward.restype = i32
+    h.swa_forward_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double,
+                                 ctypes.POINTER(i64), i32, vp]
+    h.swa_forward_ex.restype = i32
+    h.swa_band_weights.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double,
+                                   ctypes.POINTER(i64), i32, vp]
+    h.swa_band_weights.restype = i32
     h.swa_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     h.swa_decode.restype = i32
     h.swa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]

@@ -7,6 +7,11 @@
 // it, and only edge tiles are masked ("NNX Sliding-Window Attention", A local mask is not
 // a sparse implementation: only the allowed windows need computing).
 //
+// Q, K and V are read through 4-D tensor maps {D, T, H, B}, so any (b, h, t) element
+// strides the TMA unit accepts work: contiguous [B,H,T,D], or the [B,T,H,D] layout of
+// "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2). The output is
+// written with its own (b, h, t) strides.
+//
 // The grid holds at most one CTA per SM; CTA g takes items g, then 2G-1-g, then 2G+g, ...
 // of the list ordered heaviest first (a snake over the list), which balances the load
 // without any device-side queue.
@@ -85,15 +90,17 @@ __device__ __forceinline__ int pp_item(int r, int g, int G, int n) {
 }
 
 struct PPItem {
-    int bh, qt[2], f[2], l[2], k0, k1;
+    int b, h, qt[2], f[2], l[2], k0, k1;
     bool hasB;
 };
 
-__device__ __forceinline__ PPItem pp_decode(int u, int BH, int n_qt, int T, int W) {
+__device__ __forceinline__ PPItem pp_decode(int u, int BH, int H, int n_qt, int T, int W) {
     PPItem it;
     const int n_pairs = (n_qt + 1) >> 1;
     const int p = n_pairs - 1 - u / BH;  // heaviest pairs first
-    it.bh = u % BH;
+    const int bh = u % BH;
+    it.b = bh / H;
+    it.h = bh - it.b * H;
     it.qt[0] = 2 * p;
     it.qt[1] = 2 * p + 1;
     it.hasB = it.qt[1] < n_qt;
@@ -166,22 +173,35 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
 // more than the rescale threshold moves m up by the integer k = ceil(excess) and scales
 // O and l by 2^-k (exact). The row sum adds the weights exactly as written, so O is
 // normalised by the weights the MMAs multiply by.
-template <int D, bool EDGE, bool PRECISE>
+// MASK: 0 every key of the tile is in the row's band; 1 only columns cmin..cmax are; 2
+// columns cmin..cmax and cmin2..cmax2 are. before_rescale() runs (warp-uniformly) before O
+// is rescaled, for callers whose last P.V product may still be in flight.
+template <int D, int MASK, bool PRECISE, typename BeforeRescale>
 __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
-                                        float& l, int cmin, int cmax) {
+                                        float& l, int cmin, int cmax, int cmin2, int cmax2,
+                                        BeforeRescale before_rescale) {
     uint32_t v[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) ptx::tmem_ld32(scol + 32 * c, v[c]);
     ptx::tmem_ld_wait();
 #pragma unroll
     for (int c = 0; c < 4; ++c) ptx::reg_fence(v[c]);
-    if (EDGE) {
+    if (MASK == 1) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int k = 32 * c + t;
                 if (!(k >= cmin && k <= cmax)) v[c][t] = __float_as_uint(-INFINITY);
+            }
+    } else if (MASK == 2) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int k = 32 * c + t;
+                if (!((k >= cmin && k <= cmax) || (k >= cmin2 && k <= cmax2)))
+                    v[c][t] = __float_as_uint(-INFINITY);
             }
     }
     float q[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -198,6 +218,7 @@ __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scal
     if (__any_sync(0xffffffffu, need)) {
         const int k = need ? min(126, (int)ceilf(tm - m)) : 0;
         const float f = pp_pow2_neg(k);
+        before_rescale();
         __syncwarp();
         pp_rescale<D, PRECISE>(ocol, scol, 0, f);
         l *= f;
@@ -233,7 +254,8 @@ template <int D>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-                      int BH, int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
+                      int64_t osb, int64_t osh, int64_t ost, int BH, int H, int T, int W, int n_qt,
+                      float scale_log2, uint64_t wait_limit_ns,
                       int* status) {
     using C = PPCfg<D>;
     constexpr int NS = C::kStages;
@@ -300,7 +322,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
                 if (u < 0) break;
-                const PPItem it = pp_decode(u, BH, n_qt, T, W);
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (!ok || (x == 1 && !it.hasB)) break;
@@ -309,7 +331,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     uint8_t* dst = smem + C::kQOff + x * C::kTileBytes;
                     ptx::mbar_arrive_expect_tx(q_full + x, C::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
-                        ptx::tma_load_3d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.bh);
+                        ptx::tma_load_4d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.h, it.b);
                     ++nq[x];
                 }
                 for (int kt = it.k0; kt <= it.k1 && ok; ++kt) {
@@ -321,8 +343,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                         uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
                         ptx::mbar_arrive_expect_tx(ring_full + st, C::kTileBytes);
                         for (int c = 0; c < D / 64; ++c)
-                            ptx::tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, ring_full + st, c * 64,
-                                             kt * 128, it.bh);
+                            ptx::tma_load_4d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, ring_full + st, c * 64,
+                                             kt * 128, it.h, it.b);
                         ++loads;
                     }
                 }
@@ -355,7 +377,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
                 if (u < 0) break;
-                const PPItem it = pp_decode(u, BH, n_qt, T, W);
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
                 const int nx = it.hasB ? 2 : 1;
                 const bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
 #pragma unroll
@@ -443,7 +465,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int rr = 0; ok; ++rr) {
             const int u = pp_item(rr, g, G, n_items);
             if (u < 0) break;
-            const PPItem it = pp_decode(u, BH, n_qt, T, W);
+            const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
             if (x == 1 && !it.hasB) continue;
             const int qt = x ? it.qt[1] : it.qt[0];
             const int fx = x ? it.f[1] : it.f[0];
@@ -462,12 +484,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool edge = tile_class(T, W, 128, 128, qt, kt) != 2;
                 const int cmin = lo - kt * 128, cmax = hi - kt * 128;
                 const uint32_t scol = tl + C::colS(x), ocol = tl + C::colO(x);
+                // S_x(kt) complete implies PV_x(kt-1) complete: nothing to wait for
+                const auto none = [] {};
                 if (edge) {
-                    if (precise) pp_tile<D, true, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
-                    else pp_tile<D, true, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                    if (precise) pp_tile<D, 1, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
+                    else pp_tile<D, 1, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
                 } else {
-                    if (precise) pp_tile<D, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
-                    else pp_tile<D, false, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax);
+                    if (precise) pp_tile<D, 0, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
+                    else pp_tile<D, 0, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
@@ -480,7 +504,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             ptx::tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = out + ((int64_t)it.bh * T + i) * D;
+            __nv_bfloat16* orow = out + it.b * osb + it.h * osh + (int64_t)i * ost;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];

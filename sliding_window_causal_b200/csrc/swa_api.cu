@@ -19,6 +19,7 @@
 #include "plan.h"
 #include "prefill_simt.cuh"
 #include "prefill_pp.cuh"
+#include "weights.cuh"
 
 // Per-device status word: kernels record the first error here (atomicCAS from 0).
 __device__ int g_swa_status = 0;
@@ -113,6 +114,14 @@ int device_state(DeviceState** out) {
             e = cudaFuncSetAttribute(swa::prefill_simt_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::kSimtWarps * (2 * 4096 + 32) * 4);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::band_weights_kernel<float>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::kWeightWarps * 4096 * 4);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::band_weights_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::kWeightWarps * 4096 * 4);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         st.attrs_set = true;
     }
@@ -139,19 +148,40 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [BH, T, D] bf16 viewed as a 3-D tensor (D fastest), boxes of 64 columns x 128 rows,
-// 128-byte swizzle. Rows past T read as zeros; stores past T are dropped.
-int make_map(CUtensorMap* m, const void* ptr, int64_t BH, int64_t T, int64_t D) {
+// A bf16 [B, H, T, D] tensor with element strides st = (b, h, t) (D contiguous), viewed as
+// the 4-D tensor {D, T, H, B}: boxes of 64 columns x 128 rows of one (b, h), 128-byte
+// swizzle. Rows past T read as zeros.
+int make_map(CUtensorMap* m, const void* ptr, int64_t B, int64_t H, int64_t T, int64_t D,
+             const int64_t st[3]) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)(D * 2), (cuuint64_t)(T * D * 2)};
-    cuuint32_t box[3] = {64, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)(st[2] * 2), (cuuint64_t)(st[1] * 2), (cuuint64_t)(st[0] * 2)};
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SWA_OK;
+}
+
+// Element strides (b, h, t) of q, k, v and out. NULL means contiguous [B, H, T, D]. The
+// stride of a dimension of size 1 is never used to address memory; it is replaced by the
+// contiguous one so that every stride the TMA unit sees is valid.
+int read_strides(const char* fn, const int64_t* in, int n, int64_t B, int64_t H, int64_t T,
+                 int64_t D, int64_t out[][3]) {
+    const int64_t dense[3] = {H * T * D, T * D, D};
+    const int64_t size[3] = {B, H, T};
+    for (int a = 0; a < n; ++a)
+        for (int x = 0; x < 3; ++x) {
+            int64_t v = in ? in[3 * a + x] : dense[x];
+            if (v < 0 || v > (int64_t(1) << 38))
+                return fail(SWA_ERR_INVALID_ARG, "%s: stride %lld of operand %d is negative or too large",
+                            fn, (long long)v, a);
+            if (size[x] == 1) v = dense[x];
+            out[a][x] = v;
+        }
     return SWA_OK;
 }
 
@@ -221,6 +251,99 @@ void split_plan(int64_t B, int64_t H, int64_t D, int64_t W, int32_t* splits, int
     *splits = (int32_t)((W + c - 1) / c);
 }
 
+// Checks shared by the prefill entry points. OK means "go on" (B*H*T may still be 0).
+int check_sizes(const char* fn, int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, int dtype,
+                double scale) {
+    if (dtype != SWA_F32 && dtype != SWA_BF16)
+        return fail(SWA_ERR_INVALID_ARG, "%s: dtype %d is neither SWA_F32 nor SWA_BF16", fn, dtype);
+    if (W < 1) return fail(SWA_ERR_INVALID_ARG, "%s: window W=%lld must be >= 1", fn, (long long)W);
+    if (B < 0 || H < 0 || T < 0)
+        return fail(SWA_ERR_INVALID_ARG, "%s: negative size B=%lld H=%lld T=%lld", fn, (long long)B,
+                    (long long)H, (long long)T);
+    if (D < 1) return fail(SWA_ERR_INVALID_ARG, "%s: head dim D=%lld must be >= 1", fn, (long long)D);
+    if (!std::isfinite(scale)) return fail(SWA_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+    if (B > INT32_MAX || H > INT32_MAX || T > INT32_MAX || (B > 0 && H > INT32_MAX / B) ||
+        (T > 0 && B * H > INT64_MAX / T) || (B * H * T > 0 && B * H * T > INT64_MAX / D / 4))
+        return fail(SWA_ERR_UNSUPPORTED, "%s: sizes too large", fn);
+    return SWA_OK;
+}
+
+int forward_impl(const char* fn, const void* q, const void* k, const void* v, void* out, int64_t B,
+                 int64_t H, int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides,
+                 int dtype, void* stream) {
+    if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
+    if (B == 0 || H == 0 || T == 0) return success();
+    if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    int64_t st[4][3];
+    if (int rc = read_strides(fn, strides, 4, B, H, T, D, st)) return rc;
+    const int Wi = (int)(W < T ? W : T);  // W >= T is causal attention
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+
+    if (dtype == SWA_BF16) {
+        if (D != 64 && D != 128)
+            return fail(SWA_ERR_UNSUPPORTED, "%s: bf16 needs D = 64 or 128 (got %lld)", fn, (long long)D);
+        // The kernel takes the row maximum of the raw scores and scales it, which is the
+        // maximum of the scaled scores only for a positive scale.
+        if (!(scale > 0.0))
+            return fail(SWA_ERR_UNSUPPORTED, "%s: the bf16 path needs scale > 0 (got %g)", fn, scale);
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+            return fail(SWA_ERR_MISALIGNED, "%s: bf16 tensors must be 16-byte aligned", fn);
+        for (int a = 0; a < 4; ++a)
+            for (int x = 0; x < 3; ++x)
+                if (st[a][x] % 8 != 0)
+                    return fail(SWA_ERR_MISALIGNED,
+                                "%s: bf16 strides must be multiples of 8 elements (16 bytes); operand %d "
+                                "has stride %lld",
+                                fn, a, (long long)st[a][x]);
+        const int64_t BH = B * H;
+        const int n_qt = (int)((T + 127) / 128);
+        if ((int64_t)n_qt * BH > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+        CUtensorMap mq, mk, mv;
+        int rc;
+        if ((rc = make_map(&mq, q, B, H, T, D, st[0])) || (rc = make_map(&mk, k, B, H, T, D, st[1])) ||
+            (rc = make_map(&mv, v, B, H, T, D, st[2])))
+            return rc;
+        const float scale_log2 = (float)(1.4426950408889634 * scale);
+        if (!ds->pp_regs_ok)
+            return fail(SWA_ERR_UNSUPPORTED, "%s: prefill kernel was not compiled with %d registers per thread",
+                        fn, swa::kPPLaunchRegs);
+        const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
+        const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
+        auto* ob = static_cast<__nv_bfloat16*>(out);
+        if (D == 128)
+            swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], (int)BH, (int)H, (int)T, Wi, n_qt,
+                scale_log2, wait_limit(), ds->status);
+        else
+            swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], (int)BH, (int)H, (int)T, Wi, n_qt,
+                scale_log2, wait_limit(), ds->status);
+    } else {
+        if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: fp32 supports D <= 4096", fn);
+        if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
+            return fail(SWA_ERR_MISALIGNED, "%s: fp32 tensors must be 4-byte aligned", fn);
+        const int64_t nrows = B * H * T;
+        const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;
+        if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+        const size_t smem = (size_t)swa::kSimtWarps * (2 * D + 32) * sizeof(float);
+        swa::Strides sx;
+        for (int x = 0; x < 3; ++x) {
+            sx.q[x] = st[0][x];
+            sx.k[x] = st[1][x];
+            sx.v[x] = st[2][x];
+            sx.o[x] = st[3][x];
+        }
+        swa::prefill_simt_kernel<<<(unsigned)blocks, swa::kSimtWarps * 32, smem, s>>>(
+            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+            static_cast<float*>(out), sx, nrows, (int)H, (int)T, (int)D, Wi, (float)scale);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swa_forward launch");
+    return success();
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -254,65 +377,49 @@ int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W, int32_t* s
 
 int swa_forward(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t H,
                 int64_t T, int64_t D, int64_t W, int dtype, void* stream) {
-    if (dtype != SWA_F32 && dtype != SWA_BF16)
-        return fail(SWA_ERR_INVALID_ARG, "swa_forward: dtype %d is neither SWA_F32 nor SWA_BF16", dtype);
-    if (W < 1) return fail(SWA_ERR_INVALID_ARG, "swa_forward: window W=%lld must be >= 1", (long long)W);
-    if (B < 0 || H < 0 || T < 0)
-        return fail(SWA_ERR_INVALID_ARG, "swa_forward: negative size B=%lld H=%lld T=%lld",
-                    (long long)B, (long long)H, (long long)T);
-    if (D < 1) return fail(SWA_ERR_INVALID_ARG, "swa_forward: head dim D=%lld must be >= 1", (long long)D);
+    return forward_impl("swa_forward", q, k, v, out, B, H, T, D, W,
+                        D >= 1 ? 1.0 / std::sqrt((double)D) : 0.0, nullptr, dtype, stream);
+}
+
+int swa_forward_ex(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t H,
+                   int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides, int dtype,
+                   void* stream) {
+    return forward_impl("swa_forward_ex", q, k, v, out, B, H, T, D, W, scale, strides, dtype, stream);
+}
+
+int swa_band_weights(const void* q, const void* k, float* weights, int64_t B, int64_t H, int64_t T,
+                     int64_t D, int64_t W, double scale, const int64_t* strides, int dtype,
+                     void* stream) {
+    const char* fn = "swa_band_weights";
+    if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
     if (B == 0 || H == 0 || T == 0) return success();
-    if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "swa_forward: null pointer");
-    if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || T > INT32_MAX ||
-        B * H > INT64_MAX / T || B * H * T > INT64_MAX / D / 4)
-        return fail(SWA_ERR_UNSUPPORTED, "swa_forward: sizes too large");
-    const int Wi = (int)(W < T ? W : T);  // W >= T is causal attention
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!q || !k || !weights) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    const int64_t Wo = W < T ? W : T;
+    if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: D <= 4096", fn);
+    if (B * H * T > INT64_MAX / Wo / 4) return fail(SWA_ERR_UNSUPPORTED, "%s: sizes too large", fn);
+    const size_t esz = dtype == SWA_BF16 ? 2 : 4;
+    if (!aligned(q, esz) || !aligned(k, esz) || !aligned(weights, 4))
+        return fail(SWA_ERR_MISALIGNED, "%s: tensors must be aligned to their element size", fn);
+    int64_t st[2][3];
+    if (int rc = read_strides(fn, strides, 2, B, H, T, D, st)) return rc;
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
-
-    if (dtype == SWA_BF16) {
-        if (D != 64 && D != 128)
-            return fail(SWA_ERR_UNSUPPORTED, "swa_forward: bf16 needs D = 64 or 128 (got %lld)", (long long)D);
-        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
-            return fail(SWA_ERR_MISALIGNED, "swa_forward: bf16 tensors must be 16-byte aligned");
-        const int64_t BH = B * H;
-        const int n_qt = (int)((T + 127) / 128);
-        if ((int64_t)n_qt * BH > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "swa_forward: too many tiles");
-        CUtensorMap mq, mk, mv;
-        int rc;
-        if ((rc = make_map(&mq, q, BH, T, D)) || (rc = make_map(&mk, k, BH, T, D)) ||
-            (rc = make_map(&mv, v, BH, T, D)))
-            return rc;
-        const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-        if (!ds->pp_regs_ok)
-            return fail(SWA_ERR_UNSUPPORTED,
-                        "swa_forward: prefill kernel was not compiled with %d registers per thread",
-                        swa::kPPLaunchRegs);
-        const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
-        const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
-        auto* ob = static_cast<__nv_bfloat16*>(out);
-        if (D == 128)
-            swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-        else
-            swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, (int)BH, (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status);
-    } else {
-        if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "swa_forward: fp32 supports D <= 4096");
-        if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
-            return fail(SWA_ERR_MISALIGNED, "swa_forward: fp32 tensors must be 4-byte aligned");
-        const int64_t nrows = B * H * T;
-        const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;
-        if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "swa_forward: too many rows");
-        const size_t smem = (size_t)swa::kSimtWarps * (2 * D + 32) * sizeof(float);
-        const float scale = (float)(1.0 / std::sqrt((double)D));
-        swa::prefill_simt_kernel<<<(unsigned)blocks, swa::kSimtWarps * 32, smem, s>>>(
-            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-            static_cast<float*>(out), nrows, (int)T, (int)D, Wi, scale);
-    }
+    const int64_t nrows = B * H * T;
+    const int64_t blocks = (nrows + swa::kWeightWarps - 1) / swa::kWeightWarps;
+    if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+    const size_t smem = (size_t)swa::kWeightWarps * D * sizeof(float);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == SWA_BF16)
+        swa::band_weights_kernel<__nv_bfloat16><<<(unsigned)blocks, swa::kWeightWarps * 32, smem, s>>>(
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), weights,
+            st[0][0], st[0][1], st[0][2], st[1][0], st[1][1], st[1][2], nrows, (int)H, (int)T, (int)D,
+            (int)Wo, (float)scale);
+    else
+        swa::band_weights_kernel<float><<<(unsigned)blocks, swa::kWeightWarps * 32, smem, s>>>(
+            static_cast<const float*>(q), static_cast<const float*>(k), weights, st[0][0], st[0][1],
+            st[0][2], st[1][0], st[1][1], st[1][2], nrows, (int)H, (int)T, (int)D, (int)Wo, (float)scale);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "swa_forward launch");
+    if (e != cudaSuccess) return cuda_fail(e, "swa_band_weights launch");
     return success();
 }
 
