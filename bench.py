@@ -5,9 +5,11 @@
 A step is one swa_forward over the Mistral-shaped workload (B=1, H=32, T=16384,
 D=128, W=4096, bf16), inputs resident in HBM. The same run then times swa_decode over
 the streaming workload (B=64 streams, H=32, D=128, W=4096 ring, positions uniform in
-[0, 100000)) in a second timed region and reports it under "decode". Useful prefill
-FLOPs count the band only: 4*B*H*D*sum_i min(i+1, W). Decode bytes are the K/V slots
-read plus q, out and pos.
+[0, 100000)) in a second timed region and reports it under "decode", and the chunked
+streaming prefill (the same streams each taking 128 new tokens, swa_chunk_forward) in a
+third, under "chunk". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
+min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos; chunk bytes are
+the ring slots the chunk needs, its q, k, v, out, the appended rows and pos.
 
 Under torchrun each rank runs the same workload on its own GPU (weak scaling, no
 collective on the data path); times are the max over ranks. `--impl reference` times
@@ -66,6 +68,22 @@ def band_flops(B, H, T, D, W):
 def decode_bytes(B, H, D, W, pos):
     n = torch.clamp(pos + 1, max=W).sum().item()
     return int(n * H * D * 2 * 2 + 2 * B * H * D * 2 + 8 * B)
+
+
+def chunk_work(B, H, C, D, W, pos):
+    """(band FLOPs, algorithmic bytes) of one chunked streaming step: row c of stream b
+    (position P = pos[b] + c) scores min(P+1, W) keys; the bytes are the ring slots the
+    chunk needs (positions max(0, pos-W+1) .. pos-1, K and V), the chunk's q, k, v and
+    out, the appended K and V rows and pos."""
+    flops = 0
+    ring_slots = 0
+    for p in pos.tolist():
+        P = torch.arange(p, p + C, dtype=torch.int64)
+        flops += int(torch.clamp(P + 1, max=W).sum().item())
+        ring_slots += min(p, W - 1)
+    flops *= 4 * H * D
+    nbytes = H * ring_slots * D * 2 * 2 + B * H * C * D * 2 * 4 + B * H * min(C, W) * D * 2 * 2 + 8 * B
+    return flops, nbytes
 
 
 def load_peaks():
@@ -240,6 +258,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--workload", default="mistral",
                     help="prefill workload of the main line: mistral (default), small, "
                          "sweep-w{1,256,1024,4096,8192}")
@@ -335,6 +354,39 @@ def main():
             "clocks": dclk.summary(), "gpu_launches": args.steps,
         }
 
+    # ------------------------------------------------------------ chunked streaming prefill
+    chunk_line = None
+    if not args.no_chunk:
+        torch.cuda.empty_cache()
+        cw = inputs.CHUNKED
+        cq, ck, cv, ckr, cvr, cpos = inputs.for_workload(cw)
+        cflops, cbytes = chunk_work(cw.B, cw.H, cw.C, cw.D, cw.W, cpos)
+        cq, ck, cv, ckr, cvr, cpos = (t.to(device) for t in (cq, ck, cv, ckr, cvr, cpos))
+        cout = torch.empty_like(cq)
+        # Every step processes the same chunk at the same positions (the append rewrites the
+        # same slots), so every step does the same work.
+        stepc = lambda: swa.chunk_forward(cq, ck, cv, ckr, cvr, cpos, cw.W, out=cout)
+        for _ in range(args.warmup):
+            stepc()
+        swa.device_status()
+        with ClockSampler(dev_index) as cclk:
+            cms = timed(stepc, args.steps, stream, pg, device) / args.steps
+        swa.device_status()
+        cgbs = cbytes / (cms * 1e-3) / 1e9
+        ctf = cflops / (cms * 1e-3) / 1e12
+        chunk_line = {
+            "metric": "chunked streaming prefill HBM GB/s", "value": world * cgbs, "unit": "GB/s",
+            "ms_per_step": cms, "tflops": world * ctf,
+            "config": {"workload": cw.name, "B": cw.B, "H": cw.H, "C": cw.C, "D": cw.D, "W": cw.W,
+                       "pos": "uniform [0, 100000)", "seed": cw.seed, "band_flops": cflops,
+                       "l2": f"inputs larger than L2 ({2 * ckr.numel() * 2 / 1e9:.2f} GB of rings)"},
+            "roofline": {"bound": "hbm", "achieved": cgbs, "peak": peak_gbs, "unit": "GB/s",
+                         "frac": cgbs / peak_gbs, "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes": cbytes, "tensor_frac": ctf / peak_tf},
+            "clocks": cclk.summary(), "gpu_launches": 2 * args.steps,
+        }
+        del cq, ck, cv, ckr, cvr, cpos, cout
+
     # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -360,6 +412,7 @@ def main():
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
         "decode": decode_line,
+        "chunk": chunk_line,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -148,6 +148,52 @@ int swa_decode(const void* q, const void* kring, const void* vring, const int64_
                void* out, int64_t B, int64_t H, int64_t D, int64_t W, void* stream);
 
 /*
+ * swa_chunk_forward: chunked streaming prefill. C new tokens per stream attend to the
+ * rolling buffer and to each other, then join the buffer.
+ *
+ * "25. Sliding-Window Causal Attention for Streaming Inference" (Problem) processes an
+ * unbounded stream with a KV cache bounded by the window. Stream b has seen positions
+ * 0 .. pos[b]-1, and its rings hold the last min(pos[b], W) of them, position p in slot
+ * p mod W (the swa_decode layout). The chunk's tokens take positions pos[b] .. pos[b]+C-1.
+ * Chunk row c (position P = pos[b] + c) attends to positions max(0, P-W+1) .. P: those
+ * below pos[b] are read from the rings, the others from k and v. Then the chunk is
+ * appended as swa_ring_append does, so after the call the rings hold positions up to
+ * pos[b]+C-1, ready for the next chunk (pos[b] + C) or for swa_decode.
+ *
+ *   q, k, v, out : [B, H, C, D] bf16 contiguous, the chunk's queries, keys, values and
+ *                  the output.
+ *   kring, vring : [B, H, W, D] bf16 contiguous, read, then updated in place.
+ *   pos          : [B] int64 on the device: tokens stream b had before the chunk (>= 0).
+ *   D            : 64 or 128. All pointers 16-byte aligned (pos 8-byte).
+ * The attention runs on the tensor cores (tcgen05, fp32 accumulation, one rounding of the
+ * output to bf16); the append is a copy. Both are enqueued on `stream`, in that order.
+ * Errors: as swa_decode; B*H*C == 0 -> SWA_OK with nothing enqueued. A negative pos[b]
+ * is found on the device: that stream's output is written as zeros, its rings are left
+ * as they were, and swa_device_status() reports SWA_ERR_INVALID_ARG. out must not alias
+ * any input; k, v must not alias the rings.
+ */
+int swa_chunk_forward(const void* q, const void* k, const void* v, void* kring, void* vring,
+                      const int64_t* pos, void* out, int64_t B, int64_t H, int64_t C,
+                      int64_t D, int64_t W, void* stream);
+
+/*
+ * swa_ring_append: write C new tokens' keys and values into the rolling buffer.
+ *
+ * Position pos[b] + c of stream b goes to slot (pos[b] + c) mod W of kring and vring
+ * ("25. Sliding-Window Causal Attention for Streaming Inference", Problem: the cache keeps
+ * only the last W positions). When C > W only the last W tokens are written (the earlier
+ * ones would be overwritten by the same call). Use it to seed the rings after a prefill
+ * (pos = 0, C = T: the last min(T, W) positions land in their slots) or to add the token
+ * a decode step will query (C = 1, pos = that token's position) before swa_decode.
+ *   k, v         : [B, H, C, D] bf16 contiguous.  kring, vring : [B, H, W, D] bf16.
+ *   pos          : [B] int64 on the device, each >= 0.  D : 64 or 128.
+ * Errors: as swa_chunk_forward (a negative pos[b] leaves that stream's rings untouched and
+ * is reported by swa_device_status()).
+ */
+int swa_ring_append(const void* k, const void* v, void* kring, void* vring, const int64_t* pos,
+                    int64_t B, int64_t H, int64_t C, int64_t D, int64_t W, void* stream);
+
+/*
  * swa_device_status: synchronize `stream`, then read and clear the current device's
  * status word. Returns SWA_OK, or the first error a kernel recorded since the last
  * call (SWA_ERR_TIMEOUT, SWA_ERR_INVALID_ARG), or SWA_ERR_CUDA if the synchronize or

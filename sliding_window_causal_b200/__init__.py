@@ -10,6 +10,9 @@ PyTorch only supplies device memory and streams.
                                         of a [B,T,H,D] tensor
     band_weights(q, k, window)          the softmax weights of each band, [B,H,T,min(W,T)]
     decode(q, kring, vring, pos, window)  one query per stream over a W-slot ring
+    chunk_forward(q, k, v, kring, vring, pos, window)  C new tokens per stream over the
+                                        ring, then appended to it (streaming prefill)
+    ring_append(k, v, kring, vring, pos, window)       write tokens into the ring
     forward_host(...)                   prefill from pinned host tensors (copies included)
 """
 import ctypes
@@ -17,7 +20,7 @@ import ctypes
 from . import _native
 from ._native import SWA_BF16, SWA_F32, SwaError, check
 
-__all__ = ["forward", "band_weights", "decode", "forward_host", "device_status", "tile_class", "valid_slots",
+__all__ = ["forward", "band_weights", "decode", "chunk_forward", "ring_append", "forward_host", "device_status", "tile_class", "valid_slots",
            "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
 
 
@@ -142,6 +145,56 @@ def decode(q, kring, vring, pos, window, out=None):
                                        pos.data_ptr(), out.data_ptr(), B, H, D, int(window),
                                        _stream_ptr(dev)))
     return out
+
+
+def _stream_tensors(k, kring, vring, pos, window):
+    torch = _torch()
+    if k.dim() != 4 or kring.dim() != 4:
+        raise ValueError("chunk tensors must be [B,H,C,D] and the rings [B,H,W,D]")
+    B, H, C, D = k.shape
+    if kring.shape != (B, H, window, D) or vring.shape != kring.shape:
+        raise ValueError("rings must be [B,H,W,D] with W = window")
+    if pos.shape != (B,) or pos.dtype != torch.int64:
+        raise ValueError("pos must be int64 [B]")
+    if any(t.dtype != torch.bfloat16 for t in (k, kring, vring)):
+        raise TypeError("streaming calls take bf16 tensors")
+    return B, H, C, D
+
+
+def chunk_forward(q, k, v, kring, vring, pos, window, out=None):
+    """Chunked streaming prefill: q, k, v [B,H,C,D] bf16 are C new tokens per stream at
+    positions pos[b] .. pos[b]+C-1; kring, vring [B,H,W,D] hold each stream's last
+    min(pos[b], W) positions (slot = position mod W). Returns out [B,H,C,D]; afterwards
+    the rings also hold the chunk (updated in place)."""
+    torch = _torch()
+    B, H, C, D = _stream_tensors(k, kring, vring, pos, window)
+    if q.shape != k.shape or v.shape != k.shape or q.dtype != k.dtype or v.dtype != k.dtype:
+        raise ValueError("q, k, v must share one bf16 [B,H,C,D] shape")
+    dev = _need_cuda(q, k, v, kring, vring, pos)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need_cuda(out)
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_chunk_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              kring.data_ptr(), vring.data_ptr(), pos.data_ptr(),
+                                              out.data_ptr(), B, H, C, D, int(window),
+                                              _stream_ptr(dev)))
+    return out
+
+
+def ring_append(k, v, kring, vring, pos, window):
+    """Write k, v [B,H,C,D] (positions pos[b] .. pos[b]+C-1) into the rings in place,
+    position p into slot p mod W (only the last W tokens when C > W)."""
+    torch = _torch()
+    B, H, C, D = _stream_tensors(k, kring, vring, pos, window)
+    if v.shape != k.shape or v.dtype != k.dtype:
+        raise ValueError("k and v must share one bf16 [B,H,C,D] shape")
+    dev = _need_cuda(k, v, kring, vring, pos)
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_ring_append(k.data_ptr(), v.data_ptr(), kring.data_ptr(),
+                                            vring.data_ptr(), pos.data_ptr(), B, H, C, D,
+                                            int(window), _stream_ptr(dev)))
 
 
 def forward_host(q, k, v, window, out=None, device=None, staging=None):

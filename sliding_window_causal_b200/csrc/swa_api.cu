@@ -15,6 +15,7 @@
 #include <utility>
 
 #include "swa.h"
+#include "chunk.cuh"
 #include "decode.cuh"
 #include "plan.h"
 #include "prefill_simt.cuh"
@@ -100,6 +101,12 @@ int device_state(DeviceState** out) {
             e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::PPCfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::chunk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::ChunkCfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::chunk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::ChunkCfg<64>::kSmemBytes);
         if (e == cudaSuccess)
             e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e == cudaSuccess) {
@@ -464,6 +471,98 @@ int swa_decode(const void* q, const void* kring, const void* vring, const int64_
             qb, kb, vb, pos, ob, (int)H, (int)W, chunk, S, scale_log2, part, counters, ds->status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "swa_decode launch");
+    return success();
+}
+
+}  // extern "C"
+
+namespace {
+// Checks shared by the streaming entry points (chunk attention and ring append).
+int check_stream_args(const char* fn, int64_t B, int64_t H, int64_t C, int64_t D, int64_t W) {
+    if (W < 1) return fail(SWA_ERR_INVALID_ARG, "%s: window W=%lld must be >= 1", fn, (long long)W);
+    if (B < 0 || H < 0 || C < 0)
+        return fail(SWA_ERR_INVALID_ARG, "%s: negative size B=%lld H=%lld C=%lld", fn, (long long)B,
+                    (long long)H, (long long)C);
+    if (D < 1) return fail(SWA_ERR_INVALID_ARG, "%s: head dim D=%lld must be >= 1", fn, (long long)D);
+    if (B * H * C == 0) return SWA_OK;
+    if (D != 64 && D != 128)
+        return fail(SWA_ERR_UNSUPPORTED, "%s: D must be 64 or 128 (got %lld)", fn, (long long)D);
+    if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || C > INT32_MAX || W > INT32_MAX / 2 ||
+        B * H > INT64_MAX / (W > C ? W : C) / D)
+        return fail(SWA_ERR_UNSUPPORTED, "%s: sizes too large", fn);
+    return SWA_OK;
+}
+
+int launch_append(const char* fn, const void* k, const void* v, void* kring, void* vring, const int64_t* pos,
+                  int64_t B, int64_t H, int64_t C, int64_t D, int64_t W, cudaStream_t s, int* status) {
+    const int64_t c_first = C > W ? C - W : 0;
+    const int vpr = (int)(D / 8);
+    const int64_t n_vec = B * H * (C - c_first) * vpr;
+    int64_t blocks = (n_vec + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    swa::ring_append_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kring),
+        static_cast<uint4*>(vring), pos, (int)H, (int)C, (int)W, vpr, (int)c_first, n_vec, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return SWA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int swa_ring_append(const void* k, const void* v, void* kring, void* vring, const int64_t* pos, int64_t B,
+                    int64_t H, int64_t C, int64_t D, int64_t W, void* stream) {
+    const char* fn = "swa_ring_append";
+    if (int rc = check_stream_args(fn, B, H, C, D, W)) return rc;
+    if (B * H * C == 0) return success();
+    if (!k || !v || !kring || !vring || !pos) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(kring, 16) || !aligned(vring, 16) || !aligned(pos, 8))
+        return fail(SWA_ERR_MISALIGNED, "%s: tensors must be 16-byte aligned (pos 8-byte)", fn);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    if (int rc = launch_append(fn, k, v, kring, vring, pos, B, H, C, D, W, static_cast<cudaStream_t>(stream),
+                               ds->status))
+        return rc;
+    return success();
+}
+
+int swa_chunk_forward(const void* q, const void* k, const void* v, void* kring, void* vring,
+                      const int64_t* pos, void* out, int64_t B, int64_t H, int64_t C, int64_t D, int64_t W,
+                      void* stream) {
+    const char* fn = "swa_chunk_forward";
+    if (int rc = check_stream_args(fn, B, H, C, D, W)) return rc;
+    if (B * H * C == 0) return success();
+    if (!q || !k || !v || !kring || !vring || !pos || !out)
+        return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(kring, 16) || !aligned(vring, 16) ||
+        !aligned(out, 16) || !aligned(pos, 8))
+        return fail(SWA_ERR_MISALIGNED, "%s: tensors must be 16-byte aligned (pos 8-byte)", fn);
+    const int64_t n_qt = (C + 127) / 128;
+    if (B * H * n_qt > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const int64_t cst[3] = {H * C * D, C * D, D}, rst[3] = {H * W * D, W * D, D};
+    CUtensorMap mq, mk, mv, mkr, mvr;
+    int rc;
+    if ((rc = make_map(&mq, q, B, H, C, D, cst)) || (rc = make_map(&mk, k, B, H, C, D, cst)) ||
+        (rc = make_map(&mv, v, B, H, C, D, cst)) || (rc = make_map(&mkr, kring, B, H, W, D, rst)) ||
+        (rc = make_map(&mvr, vring, B, H, W, D, rst)))
+        return rc;
+    const float scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto* ob = static_cast<__nv_bfloat16*>(out);
+    const unsigned grid = (unsigned)(B * H * n_qt);
+    if (D == 128)
+        swa::chunk_kernel<128><<<grid, swa::kChunkThreads, swa::ChunkCfg<128>::kSmemBytes, s>>>(
+            mq, mk, mv, mkr, mvr, pos, ob, (int)H, (int)C, (int)W, (int)n_qt, scale_log2, wait_limit(), ds->status);
+    else
+        swa::chunk_kernel<64><<<grid, swa::kChunkThreads, swa::ChunkCfg<64>::kSmemBytes, s>>>(
+            mq, mk, mv, mkr, mvr, pos, ob, (int)H, (int)C, (int)W, (int)n_qt, scale_log2, wait_limit(), ds->status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swa_chunk_forward launch");
+    // the ring takes the chunk only after every read of the attention above (same stream)
+    if ((rc = launch_append(fn, k, v, kring, vring, pos, B, H, C, D, W, s, ds->status))) return rc;
     return success();
 }
 

@@ -5,7 +5,8 @@ arithmetic. The tests feed the same host tensors to the float64 oracle and to th
 CUDA library; the benchmark uses the same recipes.
 
 Recipe: one CPU torch.Generator per workload, seeded with 1000 + the workload's index.
-torch.randn in float32 is drawn in the order q, k, v (then the positions for decode),
+torch.randn in float32 is drawn in the order q, k, v (then the rings and positions for
+the streaming workloads),
 and rounded to bfloat16 (round to nearest even, torch's .to()) when the workload is
 bf16. Tensors larger than CHUNK elements are drawn one leading index at a time, so
 the host never holds a float32 copy of a multi-gigabyte ring.
@@ -41,6 +42,19 @@ class Decode:
     seed: int
 
 
+@dataclass(frozen=True)
+class Chunk:
+    name: str
+    B: int
+    H: int
+    C: int
+    D: int
+    W: int
+    pos_max: int
+    dtype: torch.dtype
+    seed: int
+
+
 # The five workloads, in order; seed = 1000 + index.
 TINY = [Prefill(f"tiny fp32 B1 H2 T6 D4 W{w}", 1, 2, 6, 4, w, torch.float32, 1000) for w in (3, 6, 1)]
 SMALL = Prefill("small bf16 B1 H8 T512 D64 W128", 1, 8, 512, 64, 128, torch.bfloat16, 1001)
@@ -50,6 +64,10 @@ SWEEP = [Prefill(f"window sweep bf16 B2 H16 T8192 D128 W{w}", 2, 16, 8192, 128, 
          for w in (1, 256, 1024, 4096, 8192)]
 DECODE = Decode("streaming decode bf16 B64 H32 D128 W4096", 64, 32, 128, 4096, 100000,
                 torch.bfloat16, 1004)
+# Chunked streaming prefill: the decode workload's streams and rings, each taking a chunk of
+# 128 new tokens at once instead of one (seed 1005).
+CHUNKED = Chunk("streaming chunk bf16 B64 H32 C128 D128 W4096", 64, 32, 128, 128, 4096, 100000,
+                torch.bfloat16, 1005)
 
 
 def _randn(gen, shape, dtype):
@@ -84,7 +102,22 @@ def decode_inputs(B, H, D, W, pos_max, dtype, seed):
     return q, kring, vring, pos
 
 
+def chunk_inputs(B, H, C, D, W, pos_max, dtype, seed):
+    """q, k, v [B,H,C,D] (the chunk), kring and vring [B,H,W,D] i.i.d. N(0,1) rounded to
+    dtype, and pos [B] int64 uniform in [0, pos_max), all on the CPU."""
+    gen = torch.Generator().manual_seed(seed)
+    q = _randn(gen, (B, H, C, D), dtype)
+    k = _randn(gen, (B, H, C, D), dtype)
+    v = _randn(gen, (B, H, C, D), dtype)
+    kring = _randn(gen, (B, H, W, D), dtype)
+    vring = _randn(gen, (B, H, W, D), dtype)
+    pos = torch.randint(0, pos_max, (B,), generator=gen, dtype=torch.int64)
+    return q, k, v, kring, vring, pos
+
+
 def for_workload(wl):
     if isinstance(wl, Prefill):
         return prefill_inputs(wl.B, wl.H, wl.T, wl.D, wl.dtype, wl.seed)
+    if isinstance(wl, Chunk):
+        return chunk_inputs(wl.B, wl.H, wl.C, wl.D, wl.W, wl.pos_max, wl.dtype, wl.seed)
     return decode_inputs(wl.B, wl.H, wl.D, wl.W, wl.pos_max, wl.dtype, wl.seed)

@@ -1,0 +1,180 @@
+"""Chunked streaming prefill and the ring append (swa_chunk_forward, swa_ring_append
+through the C ABI) against the float64 oracle."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_causal_b200 as swa
+from sliding_window_causal_b200 import _native, inputs
+from gpu_util import TOL, f64, max_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+BF = torch.bfloat16
+
+
+def run_chunk(q, k, v, kr, vr, pos, W):
+    """GPU chunk step on device copies; returns (out, new kring, new vring) on the host."""
+    dk, dv = kr.to(DEV), vr.to(DEV)
+    out = swa.chunk_forward(q.to(DEV), k.to(DEV), v.to(DEV), dk, dv, pos.to(DEV), W)
+    swa.device_status()
+    return out.cpu(), dk.cpu(), dv.cpu()
+
+
+def check_chunk(q, k, v, kr, vr, pos, W, tol=TOL[BF]):
+    out, nk, nv = run_chunk(q, k, v, kr, vr, pos, W)
+    ref = oracle.chunk(f64(q), f64(k), f64(v), f64(kr), f64(vr), pos.numpy(), W)
+    err = max_err(out, ref)
+    assert err <= tol, f"chunk max err {err}"
+    ek, ev = oracle.ring_append(f64(k), f64(v), f64(kr), f64(vr), pos.numpy(), W)
+    assert np.array_equal(f64(nk), ek) and np.array_equal(f64(nv), ev), "ring after the append"
+    return err
+
+
+CASES = [
+    # B, H, C, D, W, positions (one per stream)
+    (3, 2, 5, 64, 3, [0, 1, 10]),
+    (2, 2, 128, 128, 128, [0, 300]),
+    (2, 1, 129, 128, 129, [5, 1000]),
+    (3, 2, 300, 64, 200, [0, 199, 201]),
+    (2, 2, 64, 128, 1000, [0, 999]),
+    (2, 2, 1, 128, 4096, [17, 100000]),
+    (1, 2, 40, 64, 1, [77]),
+    (2, 1, 200, 128, 64, [63, 64]),
+    (1, 3, 250, 128, 1000, [4000]),
+    (2, 2, 7, 64, 127, [126, 500]),
+]
+
+
+@pytest.mark.parametrize("B,H,C,D,W,P", CASES)
+def test_chunk_matches_oracle(B, H, C, D, W, P):
+    q, k, v, kr, vr, _ = inputs.chunk_inputs(B, H, C, D, W, 1, BF, 60 + C + W)
+    check_chunk(q, k, v, kr, vr, torch.tensor(P, dtype=torch.int64), W)
+
+
+def test_stream_in_chunks_equals_prefill():
+    """A sequence fed as chunks of uneven sizes through the ring gives the rows of the
+    prefill over the whole sequence; the ring ends up holding its last W positions."""
+    B, H, T, D, W = 1, 4, 1500, 128, 300
+    q, k, v = inputs.prefill_inputs(B, H, T, D, BF, 71)
+    full = swa.forward(q.to(DEV), k.to(DEV), v.to(DEV), W).cpu()
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    dk = torch.zeros(B, H, W, D, dtype=BF, device=DEV)
+    dv = torch.zeros_like(dk)
+    p = 0
+    for c in (1, 200, 7, 300, 129, 500, T - 1137):
+        pos = torch.tensor([p], dtype=torch.int64, device=DEV)
+        out = swa.chunk_forward(q[:, :, p:p + c].contiguous().to(DEV), k[:, :, p:p + c].contiguous().to(DEV),
+                                v[:, :, p:p + c].contiguous().to(DEV), dk, dv, pos, W)
+        swa.device_status()
+        assert max_err(out, ref[:, :, p:p + c]) <= TOL[BF], f"chunk at {p}"
+        assert float((out.cpu().float() - full[:, :, p:p + c].float()).abs().max()) <= 2 * TOL[BF]
+        p += c
+    assert p == T
+    slots = [x % W for x in range(T - W, T)]
+    assert torch.equal(dk.cpu()[:, :, slots], k[:, :, T - W:]) and torch.equal(dv.cpu()[:, :, slots], v[:, :, T - W:])
+
+
+def test_one_token_chunk_and_decode_agree():
+    B, H, D, W = 4, 2, 128, 256
+    q, k, v, kr, vr, _ = inputs.chunk_inputs(B, H, 1, D, W, 1, BF, 81)
+    pos = torch.tensor([0, 5, 255, 9000], dtype=torch.int64)
+    out, nk, nv = run_chunk(q, k, v, kr, vr, pos, W)
+    dq = q[:, :, 0].contiguous().to(DEV)
+    dec = swa.decode(dq, nk.to(DEV), nv.to(DEV), pos.to(DEV), W)
+    swa.device_status()
+    ref = oracle.decode(f64(q[:, :, 0]), f64(nk), f64(nv), pos.numpy(), W)
+    assert max_err(out[:, :, 0], ref) <= TOL[BF]
+    assert max_err(dec, ref) <= TOL[BF]
+
+
+def test_ring_append_exact():
+    B, H, D, W = 2, 3, 64, 100
+    for C, P in ((1, [0, 7]), (30, [95, 3]), (250, [0, 1234]), (100, [50, 0])):
+        _, k, v, kr, vr, _ = inputs.chunk_inputs(B, H, C, D, W, 1, BF, 90 + C)
+        pos = torch.tensor(P, dtype=torch.int64)
+        dk, dv = kr.to(DEV), vr.to(DEV)
+        swa.ring_append(k.to(DEV), v.to(DEV), dk, dv, pos.to(DEV), W)
+        swa.device_status()
+        ek, ev = oracle.ring_append(f64(k), f64(v), f64(kr), f64(vr), pos.numpy(), W)
+        assert np.array_equal(f64(dk), ek) and np.array_equal(f64(dv), ev), f"C={C} pos={P}"
+
+
+def test_prefill_then_append_seeds_decode():
+    """Prefill a prompt, seed the ring from it with one append (pos 0, C = T), then decode
+    the next token: the decode output is the next prefill row."""
+    B, H, T, D, W = 1, 2, 700, 128, 256
+    q, k, v = inputs.prefill_inputs(B, H, T + 1, D, BF, 95)
+    dk = torch.zeros(B, H, W, D, dtype=BF, device=DEV)
+    dv = torch.zeros_like(dk)
+    zero = torch.zeros(B, dtype=torch.int64, device=DEV)
+    swa.ring_append(k[:, :, :T].contiguous().to(DEV), v[:, :, :T].contiguous().to(DEV), dk, dv, zero, W)
+    last = torch.full((B,), T, dtype=torch.int64, device=DEV)
+    swa.ring_append(k[:, :, T:].contiguous().to(DEV), v[:, :, T:].contiguous().to(DEV), dk, dv, last, W)
+    out = swa.decode(q[:, :, T].contiguous().to(DEV), dk, dv, last, W)
+    swa.device_status()
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)[:, :, T]
+    assert max_err(out, ref) <= TOL[BF]
+
+
+def test_negative_position_is_reported():
+    B, H, C, D, W = 3, 2, 50, 64, 64
+    q, k, v, kr, vr, _ = inputs.chunk_inputs(B, H, C, D, W, 1, BF, 97)
+    pos = torch.tensor([10, -1, 200], dtype=torch.int64)
+    dk, dv = kr.to(DEV), vr.to(DEV)
+    out = swa.chunk_forward(q.to(DEV), k.to(DEV), v.to(DEV), dk, dv, pos.to(DEV), W)
+    with pytest.raises(swa.SwaError) as e:
+        swa.device_status()
+    assert e.value.code == 1
+    assert torch.count_nonzero(out[1]) == 0
+    assert torch.equal(dk[1].cpu(), kr[1]) and torch.equal(dv[1].cpu(), vr[1])
+    good = [0, 2]
+    ref = oracle.chunk(f64(q[good]), f64(k[good]), f64(v[good]), f64(kr[good]), f64(vr[good]),
+                       pos.numpy()[good], W)
+    assert max_err(out[good], ref) <= TOL[BF]
+
+
+def test_stream_errors():
+    lib = _native.lib()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    t = torch.zeros(1, 1, 8, 64, dtype=BF, device=DEV)
+    r = torch.zeros(1, 1, 16, 64, dtype=BF, device=DEV)
+    pos = torch.zeros(1, dtype=torch.int64, device=DEV)
+    p, rp, pp = t.data_ptr(), r.data_ptr(), pos.data_ptr()
+    o = torch.empty_like(t).data_ptr()
+    f = lib.swa_chunk_forward
+    assert f(p, p, p, rp, rp, pp, o, 1, 1, 8, 64, 0, s) == 1       # W < 1
+    assert f(p, p, p, rp, rp, pp, o, 1, 1, 8, 96, 16, s) == 2      # D = 96
+    assert f(p, p, p, rp, rp, None, o, 1, 1, 8, 64, 16, s) == 1    # null pos
+    assert f(p + 2, p, p, rp, rp, pp, o, 1, 1, 8, 64, 16, s) == 3  # misaligned q
+    assert f(p, p, p, rp, rp, pp, o, 1, 1, 0, 64, 16, s) == 0      # empty chunk: no-op
+    assert f(p, p, p, rp, rp, pp, o, 1, -1, 8, 64, 16, s) == 1     # negative size
+    a = lib.swa_ring_append
+    assert a(p, p, rp, rp, pp, 1, 1, 8, 64, 0, s) == 1
+    assert a(p, p, rp, rp, pp, 1, 1, 8, 32, 16, s) == 2
+    assert a(p, p, rp + 8, rp, pp, 1, 1, 8, 64, 16, s) == 3
+    assert a(p, p, rp, rp, pp, 0, 1, 8, 64, 16, s) == 0
+    swa.device_status()
+
+
+def test_chunk_workload_full_size_sampled():
+    """The full chunked streaming workload (B64 H32 C128 D128 W4096, positions uniform
+    in [0, 100000)): every row of sampled streams against the oracle, and their rings
+    after the append bit for bit."""
+    wl = inputs.CHUNKED
+    q, k, v, kr, vr, pos = inputs.for_workload(wl)
+    dk, dv = kr.to(DEV), vr.to(DEV)
+    out = swa.chunk_forward(q.to(DEV), k.to(DEV), v.to(DEV), dk, dv, pos.to(DEV), wl.W)
+    swa.device_status()
+    for b in (0, 17, int(torch.argmin(pos)), 63):
+        for h in (0, 31):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            ref = oracle.chunk(f64(q[sl]), f64(k[sl]), f64(v[sl]), f64(kr[sl]), f64(vr[sl]),
+                               pos.numpy()[b:b + 1], wl.W)
+            assert max_err(out[sl], ref) <= TOL[BF], f"stream b={b} h={h} (pos {int(pos[b])})"
+            ek, ev = oracle.ring_append(f64(k[sl]), f64(v[sl]), f64(kr[sl]), f64(vr[sl]),
+                                        pos.numpy()[b:b + 1], wl.W)
+            assert np.array_equal(f64(dk[sl]), ek) and np.array_equal(f64(dv[sl]), ev)
