@@ -173,6 +173,35 @@ def ring_append(kc, vc, kring, vring, pos, W, lib=None):
     return kring, vring
 
 
+def mha(x, wq, bq, wk, bk, wv, bv, wo, bo, H, W, lib=None):
+    """The sliding-window multi-head attention module of "NNX Sliding-Window Attention"
+    (A complete example with moving averages), in float64: each projection is
+    y = x @ kernel + bias with a [d, d] (in x out) kernel; q, k and v are split into H
+    heads of Dh = d / H columns (head h is columns h*Dh .. h*Dh+Dh-1); every head runs
+    the sliding-window attention of forward() above; the heads are concatenated in head
+    order and projected by wo, bo. x is [B, T, d] or [T, d]; a bias may be None (zero).
+    The projections are numpy matmuls (a library step); the attention is the C oracle."""
+    x = np.asarray(x, dtype=np.float64)
+    squeeze = x.ndim == 2
+    if squeeze:
+        x = x[None]
+    B, T, d = x.shape
+    if H < 1 or d % H:
+        raise OracleError("d_model must be a multiple of the head count")
+    Dh = d // H
+
+    def linear(a, w, b):
+        y = np.matmul(a, np.asarray(w, dtype=np.float64))
+        return y if b is None else y + np.asarray(b, dtype=np.float64)
+
+    heads = lambda y: y.reshape(B, T, H, Dh).transpose(0, 2, 1, 3)
+    q, k, v = heads(linear(x, wq, bq)), heads(linear(x, wk, bk)), heads(linear(x, wv, bv))
+    o = forward(q, k, v, W, lib=lib)
+    concat = o.transpose(0, 2, 1, 3).reshape(B, T, d)
+    out = linear(concat, wo, bo)
+    return out[0] if squeeze else out
+
+
 def load_variant(path):
     """Load another build of swa_oracle.c (used by the mutation tests)."""
     return _load(path)

@@ -316,7 +316,43 @@ def pin_ring_append(lib):
                     assert np.array_equal(vr[0, h, slots], ev[slots]), f"ring v W={W} {sizes}"
 
 
+def pin_module_worked_example(lib):
+    """The module's printed example: d_model 2, two heads, window 3, zero query and key
+    kernels, identity value and output kernels, zero biases, gives the printed trailing
+    means exactly; replacing input row 0 leaves rows 3 and later unchanged."""
+    g = read_moving_average()
+    x = np.array(g["x"])
+    z, eye = np.zeros((2, 2)), np.eye(2)
+    out = oracle.mha(x, z, None, z, None, eye, None, eye, None, 2, g["W"], lib=lib)
+    assert np.array_equal(out, np.array(g["y"])), "printed module output"
+    row, vals = g["changed_row"]
+    x2 = x.copy()
+    x2[row] = vals
+    out2 = oracle.mha(x2, z, None, z, None, eye, None, eye, None, 2, g["W"], lib=lib)
+    u = g["unchanged_from"]
+    assert np.array_equal(out2[u:], out[u:])
+
+
+def pin_module_vs_torch(lib):
+    """Random kernels and biases: the module equals torch's linear layers around its
+    scaled dot-product attention with the brute-force band mask, in float64."""
+    rng = np.random.default_rng(59)
+    F = torch.nn.functional
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    for (B, T, d, H, W) in ((2, 13, 12, 3, 4), (1, 20, 8, 2, 1), (1, 9, 6, 1, 30)):
+        x = _rand(rng, B, T, d)
+        ws = [_rand(rng, d, d) / np.sqrt(d) for _ in range(4)]
+        bs = [_rand(rng, d) * 0.1 for _ in range(4)]
+        out = oracle.mha(x, ws[0], bs[0], ws[1], bs[1], ws[2], bs[2], ws[3], bs[3], H, W, lib=lib)
+        proj = [F.linear(t(x), t(ws[i]).T, t(bs[i])) for i in range(3)]
+        Dh = d // H
+        q, k, v = (p.reshape(B, T, H, Dh).transpose(1, 2) for p in proj)
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(brute.band_mask(T, W)))
+        ref = F.linear(o.transpose(1, 2).reshape(B, T, d), t(ws[3]).T, t(bs[3])).numpy()
+        assert np.abs(out - ref).max() <= TIGHT, f"module B={B} T={T} d={d} H={H} W={W}"
+
+
 ALL_PINS = [pin_band_masks, pin_moving_average, pin_trailing_mean_any_k, pin_causal_reduction,
             pin_general_band, pin_window_one, pin_independence, pin_weights, pin_rows_subset,
             pin_decode, pin_shapes, pin_scaled, pin_weights_scaled, pin_chunk_stream,
-            pin_ring_append]
+            pin_ring_append, pin_module_worked_example, pin_module_vs_torch]
