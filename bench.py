@@ -7,7 +7,8 @@ D=128, W=4096, bf16), inputs resident in HBM. The same run then times swa_decode
 the streaming workload (B=64 streams, H=32, D=128, W=4096 ring, positions uniform in
 [0, 100000)) in a second timed region and reports it under "decode", and the chunked
 streaming prefill (the same streams each taking 128 new tokens, swa_chunk_forward) in a
-third, under "chunk". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
+third, under "chunk", and the multi-head module (cuBLASLt projections around the
+attention, B1 T16384 d_model 4096, 32 heads, W4096) in a fourth, under "module". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
 min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos; chunk bytes are
 the ring slots the chunk needs, its q, k, v, out, the appended rows and pos.
 
@@ -259,6 +260,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-chunk", action="store_true")
+    ap.add_argument("--no-module", action="store_true")
     ap.add_argument("--workload", default="mistral",
                     help="prefill workload of the main line: mistral (default), small, "
                          "sweep-w{1,256,1024,4096,8192}")
@@ -387,6 +389,40 @@ def main():
         }
         del cq, ck, cv, ckr, cvr, cpos, cout
 
+    # ------------------------------------------------------------ multi-head module
+    module_line = None
+    if not args.no_module:
+        torch.cuda.empty_cache()
+        mB, mT, md, mH, mW = 1, 16384, 4096, 32, 4096
+        gm = torch.Generator().manual_seed(1006)
+        mx = torch.randn(mB, mT, md, generator=gm).to(torch.bfloat16).to(device)
+        mws = [(torch.randn(md, md, generator=gm) / md ** 0.5).to(torch.bfloat16).to(device) for _ in range(4)]
+        mbs = [(torch.randn(md, generator=gm) * 0.1).to(torch.bfloat16).to(device) for _ in range(4)]
+        mout = torch.empty_like(mx)
+        mwork = torch.empty(swa.mha_workspace_bytes(mB, mT, md, torch.bfloat16), dtype=torch.uint8, device=device)
+        mstep = lambda: swa.mha_forward(mx, mws[0], mbs[0], mws[1], mbs[1], mws[2], mbs[2], mws[3], mbs[3],
+                                        mH, mW, out=mout, workspace=mwork)
+        for _ in range(args.warmup):
+            mstep()
+        swa.device_status()
+        with ClockSampler(dev_index) as mclk:
+            mms = timed(mstep, args.steps, stream, pg, device) / args.steps
+        swa.device_status()
+        gemm_flops = 4 * 2 * mB * mT * md * md
+        attn_flops = band_flops(mB, mH, mT, md // mH, mW)
+        mtf = (gemm_flops + attn_flops) / (mms * 1e-3) / 1e12
+        module_line = {
+            "metric": "sliding-window MHA module TFLOP/s (projection + band FLOPs)", "value": world * mtf,
+            "unit": "TFLOP/s", "ms_per_step": mms,
+            "config": {"workload": f"mha module bf16 B{mB} T{mT} d{md} H{mH} W{mW}", "B": mB, "T": mT,
+                       "d_model": md, "H": mH, "W": mW, "seed": 1006, "gemm_flops": gemm_flops,
+                       "band_flops": attn_flops},
+            "roofline": {"bound": "tensor", "achieved": mtf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": mtf / peak_tf, "peak_kind": f"{peak_kind} bf16 burst", "traffic": None},
+            "clocks": mclk.summary(), "gpu_launches": args.steps,
+        }
+        del mx, mws, mbs, mout, mwork
+
     # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -413,6 +449,7 @@ def main():
         "cpu_baseline": cpu,
         "decode": decode_line,
         "chunk": chunk_line,
+        "module": module_line,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -194,6 +194,41 @@ int swa_ring_append(const void* k, const void* v, void* kring, void* vring, cons
                     int64_t B, int64_t H, int64_t C, int64_t D, int64_t W, void* stream);
 
 /*
+ * swa_mha_forward: the sliding-window multi-head attention module of "NNX Sliding-Window
+ * Attention" (A complete example with moving averages):
+ *
+ *   q = x Wq + bq, k = x Wk + bk, v = x Wv + bv   (y = x @ kernel + bias)
+ *   head h of q, k, v is columns h*Dh .. h*Dh+Dh-1, Dh = d_model / H
+ *   per head: sliding-window causal attention with window W and scale 1/sqrt(Dh)
+ *   out = concat(heads) Wo + bo
+ *
+ *   x, out       : [B, T, d_model] contiguous, of `dtype`.
+ *   wq, wk, wv, wo : [d_model, d_model] contiguous (input x output, the layout of the
+ *                  page's Linear kernels), of `dtype`.
+ *   bq, bk, bv, bo : [d_model] of `dtype`, or NULL for a zero bias.
+ *   workspace    : caller-owned device buffer of workspace_bytes >= swa_mha_workspace_bytes
+ *                  bytes, 256-byte aligned: q, k, v, the concatenated heads, and the GEMM
+ *                  library's scratch. The library allocates no device memory here.
+ *   dtype        : SWA_BF16 (Dh must be 64 or 128; projections in fp32 accumulation,
+ *                  each of q, k, v and the heads rounded once to bf16) or SWA_F32 (any
+ *                  Dh <= 4096; fp32 projections without TF32).
+ * The projections are dense GEMMs run by cuBLASLt; the attention is swa_forward_ex reading
+ * q, k, v in place as [B, T, H, Dh] (no transposes). All work is enqueued on `stream`.
+ * Errors: as swa_forward_ex, plus d_model % H != 0 or a short workspace ->
+ * SWA_ERR_INVALID_ARG, pointers not 16-byte aligned (workspace 256) -> SWA_ERR_MISALIGNED,
+ * a GEMM library failure -> SWA_ERR_CUDA. B*T == 0 -> SWA_OK with nothing enqueued.
+ */
+int swa_mha_forward(const void* x, const void* wq, const void* bq, const void* wk, const void* bk,
+                    const void* wv, const void* bv, const void* wo, const void* bo, void* out,
+                    void* workspace, int64_t workspace_bytes, int64_t B, int64_t T,
+                    int64_t d_model, int64_t H, int64_t W, int dtype, void* stream);
+
+/* swa_mha_workspace_bytes: bytes of workspace swa_mha_forward needs for these sizes
+ * (4 * B*T*d_model elements, each part rounded up to 256 bytes, plus 32 MiB of GEMM
+ * scratch), or -1 for invalid sizes or dtype. */
+int64_t swa_mha_workspace_bytes(int64_t B, int64_t T, int64_t d_model, int dtype);
+
+/*
  * swa_device_status: synchronize `stream`, then read and clear the current device's
  * status word. Returns SWA_OK, or the first error a kernel recorded since the last
  * call (SWA_ERR_TIMEOUT, SWA_ERR_INVALID_ARG), or SWA_ERR_CUDA if the synchronize or

@@ -13,6 +13,9 @@ PyTorch only supplies device memory and streams.
     chunk_forward(q, k, v, kring, vring, pos, window)  C new tokens per stream over the
                                         ring, then appended to it (streaming prefill)
     ring_append(k, v, kring, vring, pos, window)       write tokens into the ring
+    mha_forward(x, wq, bq, wk, bk, wv, bv, wo, bo, num_heads, window)
+                                        the multi-head module: projections (cuBLASLt)
+                                        around the attention
     forward_host(...)                   prefill from pinned host tensors (copies included)
 """
 import ctypes
@@ -20,7 +23,8 @@ import ctypes
 from . import _native
 from ._native import SWA_BF16, SWA_F32, SwaError, check
 
-__all__ = ["forward", "band_weights", "decode", "chunk_forward", "ring_append", "forward_host", "device_status", "tile_class", "valid_slots",
+__all__ = ["forward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
+           "mha_workspace_bytes", "forward_host", "device_status", "tile_class", "valid_slots",
            "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
 
 
@@ -195,6 +199,50 @@ def ring_append(k, v, kring, vring, pos, window):
         check(_native.lib().swa_ring_append(k.data_ptr(), v.data_ptr(), kring.data_ptr(),
                                             vring.data_ptr(), pos.data_ptr(), B, H, C, D,
                                             int(window), _stream_ptr(dev)))
+
+
+def mha_workspace_bytes(B, T, d_model, dtype):
+    """Bytes of device workspace mha_forward needs."""
+    torch = _torch()
+    code = SWA_BF16 if dtype == torch.bfloat16 else SWA_F32
+    return int(_native.lib().swa_mha_workspace_bytes(B, T, d_model, code))
+
+
+def mha_forward(x, wq, bq, wk, bk, wv, bv, wo, bo, num_heads, window, out=None, workspace=None):
+    """Sliding-window multi-head attention module: x [B,T,d] (or [T,d]); kernels [d,d]
+    (input x output); biases [d] or None; all bf16 (head width d/num_heads of 64 or 128)
+    or fp32. Returns out shaped like x. workspace: optional preallocated uint8 CUDA
+    tensor of at least mha_workspace_bytes(...) bytes."""
+    torch = _torch()
+    squeeze = x.dim() == 2
+    if squeeze:
+        x = x.unsqueeze(0)
+    if x.dim() != 3:
+        raise ValueError("x must be [B,T,d] or [T,d]")
+    B, T, d = x.shape
+    mats = [wq, wk, wv, wo]
+    biases = [bq, bk, bv, bo]
+    if any(w.shape != (d, d) for w in mats) or any(b is not None and b.shape != (d,) for b in biases):
+        raise ValueError("kernels must be [d,d] and biases [d]")
+    if any(t.dtype != x.dtype for t in mats + [b for b in biases if b is not None]):
+        raise TypeError("x, kernels and biases must share one dtype")
+    dev = _need_cuda(x, *mats, *[b for b in biases if b is not None])
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need_cuda(out)
+        out = out.view(B, T, d)
+    need = mha_workspace_bytes(B, T, d, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_mha_forward(x.data_ptr(), ptr(wq), ptr(bq), ptr(wk), ptr(bk), ptr(wv),
+                                            ptr(bv), ptr(wo), ptr(bo), out.data_ptr(),
+                                            workspace.data_ptr(), workspace.numel(), B, T, d,
+                                            int(num_heads), int(window), _dtype_code(x),
+                                            _stream_ptr(dev)))
+    return out[0] if squeeze else out
 
 
 def forward_host(q, k, v, window, out=None, device=None, staging=None):

@@ -11,13 +11,15 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "_swa.so")
-SOURCES = [os.path.join(CSRC, "swa_api.cu")]
+SOURCES = [os.path.join(CSRC, "swa_api.cu"), os.path.join(CSRC, "module.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "swa.h")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
     "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
 ]
+# cuBLASLt serves the module's projection GEMMs (swa_mha_forward)
+LINK_FLAGS = ["-lcublasLt", "-Xlinker", "-rpath", "-Xlinker", "/usr/local/cuda/lib64"]
 
 
 def nvcc():
@@ -38,7 +40,7 @@ def build(force=False, verbose=False, out=LIB, extra=()):
     """Compile the library if any source is newer than it. Returns the .so path."""
     if not force and up_to_date(out):
         return out
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", out]
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, *SOURCES, *LINK_FLAGS, "-o", out]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)

@@ -15,6 +15,7 @@
 #include <utility>
 
 #include "swa.h"
+#include "api_internal.h"
 #include "chunk.cuh"
 #include "decode.cuh"
 #include "plan.h"
@@ -699,3 +700,14 @@ extern "C" int swa_decode_noalloc(const void* q, const void* kring, const void* 
     if (e != cudaSuccess) return cuda_fail(e, "swa_decode_noalloc launch");
     return success();
 }
+
+namespace swa_internal {
+int set_error(int code, const char* msg) {
+    t_error = msg;
+    return code;
+}
+int clear_error() {
+    t_error.clear();
+    return SWA_OK;
+}
+}  // namespace swa_internal
