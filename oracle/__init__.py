@@ -35,10 +35,11 @@ def _load(path=None):
     lib.swa_oracle_forward_scaled.argtypes = [d, d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
     lib.swa_oracle_weights_scaled.argtypes = [d, d, d, i64, i64, i64, i64, i64, ctypes.c_double]
     lib.swa_oracle_chunk.argtypes = [d, d, d, d, d, pi64, d, i64, i64, i64, i64, i64]
+    lib.swa_oracle_backward.argtypes = [d, d, d, d, d, d, d, i64, i64, i64, i64, i64]
     lib.swa_oracle_ring_append.argtypes = [d, d, d, d, pi64, i64, i64, i64, i64, i64]
     for f in (lib.swa_oracle_forward, lib.swa_oracle_forward_rows, lib.swa_oracle_weights,
               lib.swa_oracle_decode, lib.swa_oracle_forward_scaled, lib.swa_oracle_weights_scaled,
-              lib.swa_oracle_chunk, lib.swa_oracle_ring_append):
+              lib.swa_oracle_chunk, lib.swa_oracle_ring_append, lib.swa_oracle_backward):
         f.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -171,6 +172,25 @@ def ring_append(kc, vc, kring, vring, pos, W, lib=None):
     if rc != 0:
         raise OracleError(f"oracle ring_append rejected its arguments (rc={rc})")
     return kring, vring
+
+
+def backward(q, k, v, dout, W, lib=None):
+    """Gradients (dq, dk, dv), each [B,H,T,D] float64, of the prefill output with respect
+    to q, k and v, given the output gradient dout [B,H,T,D]."""
+    lib = lib or _load()
+    q, pq = _f64(q)
+    k, pk = _f64(k)
+    v, pv = _f64(v)
+    dout, pdo = _f64(dout)
+    if q.ndim != 4 or any(t.shape != q.shape for t in (k, v, dout)):
+        raise OracleError("q, k, v, dout must share one [B,H,T,D] shape")
+    B, H, T, D = q.shape
+    grads = [np.empty_like(q) for _ in range(3)]
+    ptrs = [_f64(g)[1] for g in grads]
+    rc = lib.swa_oracle_backward(pq, pk, pv, pdo, *ptrs, B, H, T, D, int(W))
+    if rc != 0:
+        raise OracleError(f"oracle backward rejected its arguments (rc={rc})")
+    return tuple(grads)
 
 
 def mha(x, wq, bq, wk, bk, wv, bv, wo, bo, H, W, lib=None):

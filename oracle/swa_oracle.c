@@ -350,3 +350,94 @@ int swa_oracle_ring_append(const double* kc, const double* vc, double* kring, do
     }
     return ORACLE_OK;
 }
+
+/* Backward pass: the gradients of the prefill definition with respect to q, k and v,
+ * given the gradient dout of the output ("NNX Sliding-Window Attention", Mask before
+ * softmax: with the band masked to -inf before the softmax, the gradients are well
+ * defined for finite allowed scores). They follow from the chain rule through the
+ * definition above, row by row, with c = 1/sqrt(D):
+ *
+ *   p_j   = e_j / sum_l e_l                     for j in band(i)   (the forward weights)
+ *   dv_j += p_j * dout_i
+ *   dp_j  = dout_i . v_j
+ *   ds_j  = p_j * (dp_j - sum_l p_l dp_l)       (softmax Jacobian)
+ *   dq_i  = c * sum_j ds_j k_j
+ *   dk_j += c * ds_j q_i
+ *
+ * Keys outside band(i) receive nothing from row i. Layout and loop order as the forward;
+ * rows i ascending within each (b,h), so every sum has one fixed order. q, k, v, dout,
+ * dq, dk, dv: [B,H,T,D]. */
+int swa_oracle_backward(const double* q, const double* k, const double* v, const double* dout,
+                        double* dq, double* dk, double* dv,
+                        int64_t B, int64_t H, int64_t T, int64_t D, int64_t W) {
+    if (check_sizes(B, H, T, D, W) != ORACLE_OK) return ORACLE_INVALID;
+    if (B * H * T == 0) return ORACLE_OK;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORACLE_INVALID;
+    const int64_t band_max = (W < T) ? W : T;
+    const double c = 1.0 / sqrt((double)D);
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* p = (double*)malloc((size_t)band_max * sizeof(double));
+        double* dp = (double*)malloc((size_t)band_max * sizeof(double));
+        if (!p || !dp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bh = 0; bh < B * H; ++bh) {
+                const double* qh = q + bh * T * D;
+                const double* kh = k + bh * T * D;
+                const double* vh = v + bh * T * D;
+                const double* doh = dout + bh * T * D;
+                double* dqh = dq + bh * T * D;
+                double* dkh = dk + bh * T * D;
+                double* dvh = dv + bh * T * D;
+                for (int64_t x = 0; x < T * D; ++x) {
+                    dkh[x] = 0.0;
+                    dvh[x] = 0.0;
+                }
+                for (int64_t i = 0; i < T; ++i) {
+                    int64_t lo = i - W + 1;
+                    if (lo < 0) lo = 0;
+                    const double* qi = qh + i * D;
+                    const double* doi = doh + i * D;
+                    /* forward weights of row i */
+                    double m = -INFINITY;
+                    for (int64_t j = lo; j <= i; ++j) {
+                        double dot = 0.0;
+                        for (int64_t d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
+                        p[j - lo] = dot * c;
+                        if (p[j - lo] > m) m = p[j - lo];
+                    }
+                    double denom = 0.0;
+                    for (int64_t j = lo; j <= i; ++j) {
+                        p[j - lo] = exp(p[j - lo] - m);
+                        denom += p[j - lo];
+                    }
+                    for (int64_t j = lo; j <= i; ++j) p[j - lo] = p[j - lo] / denom;
+                    /* dp_j and the weighted sum of dp */
+                    double pdp = 0.0;
+                    for (int64_t j = lo; j <= i; ++j) {
+                        double dot = 0.0;
+                        for (int64_t d = 0; d < D; ++d) dot += doi[d] * vh[j * D + d];
+                        dp[j - lo] = dot;
+                        pdp += p[j - lo] * dot;
+                    }
+                    for (int64_t d = 0; d < D; ++d) dqh[i * D + d] = 0.0;
+                    for (int64_t j = lo; j <= i; ++j) {
+                        const double ds = p[j - lo] * (dp[j - lo] - pdp);
+                        for (int64_t d = 0; d < D; ++d) {
+                            dqh[i * D + d] += c * ds * kh[j * D + d];
+                            dkh[j * D + d] += c * ds * qi[d];
+                            dvh[j * D + d] += p[j - lo] * doi[d];
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+    }
+    return bad ? ORACLE_INVALID : ORACLE_OK;
+}

@@ -352,7 +352,47 @@ def pin_module_vs_torch(lib):
         assert np.abs(out - ref).max() <= TIGHT, f"module B={B} T={T} d={d} H={H} W={W}"
 
 
+def pin_backward_autograd(lib):
+    """The gradients equal torch autograd through its scaled dot-product attention with
+    the brute-force band mask, in float64, for several windows including W = 1 and
+    W >= T."""
+    rng = np.random.default_rng(61)
+    for (B, H, T, D, W) in ((1, 2, 9, 4, 3), (2, 1, 17, 6, 5), (1, 2, 12, 3, 1), (1, 1, 10, 5, 40)):
+        q, k, v, do = (_rand(rng, B, H, T, D) for _ in range(4))
+        dq, dk, dv = oracle.backward(q, k, v, do, W, lib=lib)
+        tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+        out = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk, tv, attn_mask=torch.from_numpy(brute.band_mask(T, W)))
+        out.backward(torch.from_numpy(do))
+        for name, a, b in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+            assert np.abs(a - b.numpy()).max() <= TIGHT, f"{name} T={T} W={W}"
+
+
+def pin_backward_finite_differences(lib):
+    """Central differences of the forward oracle (a different code path) in random
+    directions agree with the directional derivative sum(dout * d out) given by the
+    gradients."""
+    rng = np.random.default_rng(67)
+    B, H, T, D, W = 1, 2, 11, 4, 4
+    q, k, v, do = (_rand(rng, B, H, T, D) for _ in range(4))
+    grads = oracle.backward(q, k, v, do, W, lib=lib)
+    h = 1e-5
+    for which in range(3):
+        for _ in range(3):
+            u = _rand(rng, B, H, T, D)
+            args = [q, k, v]
+            plus = list(args)
+            minus = list(args)
+            plus[which] = args[which] + h * u
+            minus[which] = args[which] - h * u
+            fd = (np.sum(do * oracle.forward(*plus, W, lib=lib)) -
+                  np.sum(do * oracle.forward(*minus, W, lib=lib))) / (2 * h)
+            an = np.sum(grads[which] * u)
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), f"finite differences, operand {which}"
+
+
 ALL_PINS = [pin_band_masks, pin_moving_average, pin_trailing_mean_any_k, pin_causal_reduction,
             pin_general_band, pin_window_one, pin_independence, pin_weights, pin_rows_subset,
             pin_decode, pin_shapes, pin_scaled, pin_weights_scaled, pin_chunk_stream,
-            pin_ring_append, pin_module_worked_example, pin_module_vs_torch]
+            pin_ring_append, pin_module_worked_example, pin_module_vs_torch, pin_backward_autograd,
+            pin_backward_finite_differences]

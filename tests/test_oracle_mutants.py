@@ -48,6 +48,11 @@ MUTANTS = [
      [("int64_t first = P - W + 1;\n    if (first < 0) first = 0;\n    const double inv_sqrt_d = 1.0 / sqrt((double)D);\n    double m = -INFINITY;\n    for (int64_t p = first; p <= P; ++p) {\n        const double* kp = (p < pos0)",
        "int64_t first = P - W;\n    if (first < 0) first = 0;\n    const double inv_sqrt_d = 1.0 / sqrt((double)D);\n    double m = -INFINITY;\n    for (int64_t p = first; p <= P; ++p) {\n        const double* kp = (p < pos0)")] + WIDER_SCRATCH),
     ("ring append one slot late", [("(pos[b] + c) % W", "(pos[b] + c + 1) % W")]),
+    ("backward drops the softmax Jacobian's mean term",
+     [("const double ds = p[j - lo] * (dp[j - lo] - pdp);", "const double ds = p[j - lo] * dp[j - lo];")]),
+    ("backward dk without the scale",
+     [("dkh[j * D + d] += c * ds * qi[d];", "dkh[j * D + d] += ds * qi[d];")]),
+    ("backward dv weighted by ds", [("dvh[j * D + d] += p[j - lo] * doi[d];", "dvh[j * D + d] += ds * doi[d];")]),
     ("weights unnormalised", [("wrow[j] = wrow[j] / denom;", "wrow[j] = wrow[j];")]),
 ]
 
