@@ -8,7 +8,8 @@ the streaming workload (B=64 streams, H=32, D=128, W=4096 ring, positions unifor
 [0, 100000)) in a second timed region and reports it under "decode", and the chunked
 streaming prefill (the same streams each taking 128 new tokens, swa_chunk_forward) in a
 third, under "chunk", and the multi-head module (cuBLASLt projections around the
-attention, B1 T16384 d_model 4096, 32 heads, W4096) in a fourth, under "module". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
+attention, B1 T16384 d_model 4096, 32 heads, W4096) in a fourth, under "module", and the
+backward of the Mistral-shaped prefill in a fifth, under "backward". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
 min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos; chunk bytes are
 the ring slots the chunk needs, its q, k, v, out, the appended rows and pos.
 
@@ -39,13 +40,16 @@ L2_BYTES = 126 * 2**20
 # (dram__bytes_read.sum + dram__bytes_write.sum; the captures are summarised in profiles/).
 # Reported only while the kernel's sources are unchanged since the capture.
 KERNEL_SOURCES = {"prefill": ["prefill_pp.cuh", "ptx.cuh", "umma.h", "plan.h"],
-                  "decode": ["decode.cuh", "ptx.cuh"]}
+                  "decode": ["decode.cuh", "ptx.cuh"],
+                  "chunk": ["chunk.cuh", "prefill_pp.cuh", "ptx.cuh", "umma.h", "plan.h"]}
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
-    "prefill": {"bytes": 1103.0e6 + 115.1e6, "sources": "1afd5d34227b9f04"},
+    "prefill": {"bytes": 1146.4e6 + 114.9e6, "sources": "6b470bb70d98cbe4"},
     # 16 of the 64 streams captured (1.07 GB of rings), scaled x4 by streams: each stream
     # reads only its own ring, so traffic grows in proportion
-    "decode": {"bytes": 4 * (951.0e6 + 4.3e6), "sources": "0f022f18ed33daaa"},
+    "decode": {"bytes": 4 * (951.0e6 + 3.5e6), "sources": "e235f49578c120e3"},
+    # chunk_kernel, 16 of the 64 streams captured, scaled x4 by streams as for decode
+    "chunk": {"bytes": 4 * (1105.4e6 + 18.0e6), "sources": "d3b9c8a46ed57e86"},
 }
 
 
@@ -261,6 +265,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--no-module", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--chunk-streams", type=int, default=None,
+                    help="override the chunk workload's stream count (smaller profiling runs)")
     ap.add_argument("--workload", default="mistral",
                     help="prefill workload of the main line: mistral (default), small, "
                          "sweep-w{1,256,1024,4096,8192}")
@@ -361,6 +368,10 @@ def main():
     if not args.no_chunk:
         torch.cuda.empty_cache()
         cw = inputs.CHUNKED
+        if args.chunk_streams:
+            import dataclasses
+            cw = dataclasses.replace(cw, B=args.chunk_streams,
+                                     name=cw.name.replace("B64", f"B{args.chunk_streams}"))
         cq, ck, cv, ckr, cvr, cpos = inputs.for_workload(cw)
         cflops, cbytes = chunk_work(cw.B, cw.H, cw.C, cw.D, cw.W, cpos)
         cq, ck, cv, ckr, cvr, cpos = (t.to(device) for t in (cq, ck, cv, ckr, cvr, cpos))
@@ -383,7 +394,8 @@ def main():
                        "pos": "uniform [0, 100000)", "seed": cw.seed, "band_flops": cflops,
                        "l2": f"inputs larger than L2 ({2 * ckr.numel() * 2 / 1e9:.2f} GB of rings)"},
             "roofline": {"bound": "hbm", "achieved": cgbs, "peak": peak_gbs, "unit": "GB/s",
-                         "frac": cgbs / peak_gbs, "peak_kind": peak_kind, "traffic": None,
+                         "frac": cgbs / peak_gbs, "peak_kind": peak_kind,
+                         "traffic": measured_traffic("chunk") if cw.B == 64 else None,
                          "algorithmic_bytes": cbytes, "tensor_frac": ctf / peak_tf},
             "clocks": cclk.summary(), "gpu_launches": 2 * args.steps,
         }
@@ -423,6 +435,37 @@ def main():
         }
         del mx, mws, mbs, mout, mwork
 
+    # ------------------------------------------------------------ backward (gradients)
+    backward_line = None
+    if not args.no_backward:
+        torch.cuda.empty_cache()
+        bw = inputs.MISTRAL
+        bq, bk, bv = (t.to(device) for t in inputs.for_workload(bw))
+        gb = torch.Generator().manual_seed(1007)
+        bdo = torch.randn(bw.B, bw.H, bw.T, bw.D, generator=gb).to(bw.dtype).to(device)
+        bsteps = max(3, args.steps // 5)
+        bstep = lambda: swa.backward(bq, bk, bv, bdo, bw.W)
+        for _ in range(3):
+            bstep()
+        swa.device_status()
+        with ClockSampler(dev_index) as bclk:
+            bms = timed(bstep, bsteps, stream, pg, device) / bsteps
+        swa.device_status()
+        bflops = 5 * band_flops(bw.B, bw.H, bw.T, bw.D, bw.W) // 2  # five band products
+        btf = bflops / (bms * 1e-3) / 1e12
+        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FFMA TFLOP/s: SMs x lanes x 2 x max clock
+        backward_line = {
+            "metric": "backward TFLOP/s (2.5 x band FLOPs)", "value": world * btf, "unit": "TFLOP/s",
+            "ms_per_step": bms, "steps": bsteps,
+            "config": {"workload": bw.name + " backward", "B": bw.B, "H": bw.H, "T": bw.T, "D": bw.D,
+                       "W": bw.W, "seed": bw.seed, "dout_seed": 1007, "useful_flops": bflops},
+            "roofline": {"bound": "alu", "achieved": btf, "peak": alu_peak, "unit": "TFLOP/s",
+                         "frac": btf / alu_peak, "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                         "traffic": None},
+            "clocks": bclk.summary(), "gpu_launches": 2 * bsteps,
+        }
+        del bq, bk, bv, bdo
+
     # ------------------------------------------------------------ CPU baseline (rank 0, N = 1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -450,6 +493,7 @@ def main():
         "decode": decode_line,
         "chunk": chunk_line,
         "module": module_line,
+        "backward": backward_line,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -229,6 +229,35 @@ int swa_mha_forward(const void* x, const void* wq, const void* bq, const void* w
 int64_t swa_mha_workspace_bytes(int64_t B, int64_t T, int64_t d_model, int dtype);
 
 /*
+ * swa_backward: gradients of the prefill with respect to q, k and v.
+ *
+ * "NNX Sliding-Window Attention" (Mask before softmax) notes that with the band masked to
+ * -inf before the softmax the gradients stay well defined. With c = scale and p the
+ * forward weights (only band pairs 0 <= i-j < W take part):
+ *   dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - delta_i),
+ *   delta_i = sum_j p_ij (dout_i . v_j),  dq_i = c sum_j ds_ij k_j,  dk_j = c sum_i ds_ij q_i.
+ *   q, k, v, dout : [B,H,T,D] contiguous inputs of `dtype` (dout = dL/dout).
+ *   dq, dk, dv    : [B,H,T,D] contiguous outputs of `dtype` (overwritten).
+ *   workspace     : caller-owned device buffer of workspace_bytes >=
+ *                   swa_backward_workspace_bytes(B,H,T) bytes, 8-byte aligned: the per-row
+ *                   log-sum-exp and delta the two kernels pass along.
+ *   scale         : the forward's score scale (1/sqrt(D) for swa_forward), finite.
+ *   dtype         : SWA_F32 or SWA_BF16; the arithmetic is fp32 on the CUDA cores in both
+ *                   cases (bf16 operands are widened, bf16 gradients rounded once).
+ *   D             : 1 .. 2048.
+ * The row statistics are recomputed from q and k (no forward state is needed). There are
+ * no atomics: the results are deterministic. Errors: as swa_forward_ex, plus a short
+ * workspace -> SWA_ERR_INVALID_ARG.
+ */
+int swa_backward(const void* q, const void* k, const void* v, const void* dout,
+                 void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+                 int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, double scale,
+                 int dtype, void* stream);
+
+/* swa_backward_workspace_bytes: B*H*T*8, or -1 for negative or overflowing sizes. */
+int64_t swa_backward_workspace_bytes(int64_t B, int64_t H, int64_t T);
+
+/*
  * swa_device_status: synchronize `stream`, then read and clear the current device's
  * status word. Returns SWA_OK, or the first error a kernel recorded since the last
  * call (SWA_ERR_TIMEOUT, SWA_ERR_INVALID_ARG), or SWA_ERR_CUDA if the synchronize or

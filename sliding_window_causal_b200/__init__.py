@@ -16,6 +16,7 @@ PyTorch only supplies device memory and streams.
     mha_forward(x, wq, bq, wk, bk, wv, bv, wo, bo, num_heads, window)
                                         the multi-head module: projections (cuBLASLt)
                                         around the attention
+    backward(q, k, v, dout, window)     (dq, dk, dv) of the prefill
     forward_host(...)                   prefill from pinned host tensors (copies included)
 """
 import ctypes
@@ -23,7 +24,7 @@ import ctypes
 from . import _native
 from ._native import SWA_BF16, SWA_F32, SwaError, check
 
-__all__ = ["forward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
+__all__ = ["forward", "backward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
            "mha_workspace_bytes", "forward_host", "device_status", "tile_class", "valid_slots",
            "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
 
@@ -102,6 +103,28 @@ def forward(q, k, v, window, out=None, scale=None):
                                      B, H, T, D, int(window), sc, _bht_strides(q, k, v, out),
                                      _dtype_code(q), _stream_ptr(dev)))
     return out.squeeze(1) if squeeze else out
+
+
+def backward(q, k, v, dout, window, scale=None):
+    """Gradients (dq, dk, dv) of the prefill output with respect to q, k, v, given the
+    output gradient dout. All [B,H,T,D] contiguous CUDA tensors of one dtype (fp32 or
+    bf16, D <= 2048); fp32 arithmetic on the CUDA cores. scale defaults to 1/sqrt(D)."""
+    torch = _torch()
+    if q.dim() != 4 or any(t.shape != q.shape for t in (k, v, dout)):
+        raise ValueError("q, k, v, dout must share one [B,H,T,D] shape")
+    if any(t.dtype != q.dtype for t in (k, v, dout)):
+        raise TypeError("q, k, v, dout must share one dtype")
+    dev = _need_cuda(q, k, v, dout)
+    B, H, T, D = q.shape
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    lib = _native.lib()
+    ws = torch.empty(max(1, int(lib.swa_backward_workspace_bytes(B, H, T))), dtype=torch.uint8, device=dev)
+    sc = 1.0 / D ** 0.5 if scale is None else float(scale)
+    with torch.cuda.device(dev):
+        check(lib.swa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                               dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, H, T, D,
+                               int(window), sc, _dtype_code(q), _stream_ptr(dev)))
+    return dq, dk, dv
 
 
 def band_weights(q, k, window, scale=None):

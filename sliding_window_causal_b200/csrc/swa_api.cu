@@ -16,6 +16,7 @@
 
 #include "swa.h"
 #include "api_internal.h"
+#include "backward.cuh"
 #include "chunk.cuh"
 #include "decode.cuh"
 #include "plan.h"
@@ -79,6 +80,18 @@ struct DeviceState {
 };
 std::map<int, DeviceState> g_dev;
 
+constexpr int kBwdMaxD = 2048;
+
+template <typename TIn>
+cudaError_t set_bwd_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(swa::bwd_rows_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         swa::kBwdWarps * (3 * kBwdMaxD + 64) * 4);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(swa::bwd_cols_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 swa::kBwdWarps * (4 * kBwdMaxD + 64) * 4);
+    return e;
+}
+
 int device_state(DeviceState** out) {
     int dev;
     cudaError_t e = cudaGetDevice(&dev);
@@ -102,6 +115,8 @@ int device_state(DeviceState** out) {
             e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::PPCfg<64>::kSmemBytes);
+        if (e == cudaSuccess) e = set_bwd_attrs<float>();
+        if (e == cudaSuccess) e = set_bwd_attrs<__nv_bfloat16>();
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::chunk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::ChunkCfg<128>::kSmemBytes);
@@ -564,6 +579,63 @@ int swa_chunk_forward(const void* q, const void* k, const void* v, void* kring, 
     if (e != cudaSuccess) return cuda_fail(e, "swa_chunk_forward launch");
     // the ring takes the chunk only after every read of the attention above (same stream)
     if ((rc = launch_append(fn, k, v, kring, vring, pos, B, H, C, D, W, s, ds->status))) return rc;
+    return success();
+}
+
+int64_t swa_backward_workspace_bytes(int64_t B, int64_t H, int64_t T) {
+    if (B < 0 || H < 0 || T < 0) return -1;
+    if (B > 0 && H > 0 && T > 0 && (B * H > INT64_MAX / T || B * H * T > INT64_MAX / 8)) return -1;
+    return B * H * T * 8;
+}
+
+int swa_backward(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
+                 void* workspace, int64_t workspace_bytes, int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                 double scale, int dtype, void* stream) {
+    const char* fn = "swa_backward";
+    if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
+    if (B == 0 || H == 0 || T == 0) return success();
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace)
+        return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (workspace_bytes < swa_backward_workspace_bytes(B, H, T))
+        return fail(SWA_ERR_INVALID_ARG, "%s: workspace of %lld bytes, %lld needed", fn, (long long)workspace_bytes,
+                    (long long)swa_backward_workspace_bytes(B, H, T));
+    if (D > kBwdMaxD) return fail(SWA_ERR_UNSUPPORTED, "%s: D <= %d", fn, kBwdMaxD);
+    const size_t esz = dtype == SWA_BF16 ? 2 : 4;
+    const void* ptrs[] = {q, k, v, dout, dq, dk, dv};
+    for (const void* p : ptrs)
+        if (!aligned(p, esz)) return fail(SWA_ERR_MISALIGNED, "%s: tensors must be aligned to their element size", fn);
+    if (!aligned(workspace, 8)) return fail(SWA_ERR_MISALIGNED, "%s: workspace must be 8-byte aligned", fn);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const int64_t nrows = B * H * T;
+    const int64_t blocks = (nrows + swa::kBwdWarps - 1) / swa::kBwdWarps;
+    if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+    const int Wi = (int)(W < T ? W : T);
+    const size_t smem_rows = (size_t)swa::kBwdWarps * (3 * D + 64) * 4;
+    const size_t smem_cols = (size_t)swa::kBwdWarps * (4 * D + 64) * 4;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* stats = static_cast<float*>(workspace);
+    const float c = (float)scale;
+    if (dtype == SWA_BF16) {
+        using T16 = __nv_bfloat16;
+        swa::bwd_rows_kernel<T16><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_rows, s>>>(
+            static_cast<const T16*>(q), static_cast<const T16*>(k), static_cast<const T16*>(v),
+            static_cast<const T16*>(dout), static_cast<T16*>(dq), stats, nrows, (int)T, (int)D, Wi, c);
+        swa::bwd_cols_kernel<T16><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_cols, s>>>(
+            static_cast<const T16*>(q), static_cast<const T16*>(k), static_cast<const T16*>(v),
+            static_cast<const T16*>(dout), stats, static_cast<T16*>(dk), static_cast<T16*>(dv), nrows, (int)T,
+            (int)D, Wi, c);
+    } else {
+        swa::bwd_rows_kernel<float><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_rows, s>>>(
+            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+            static_cast<const float*>(dout), static_cast<float*>(dq), stats, nrows, (int)T, (int)D, Wi, c);
+        swa::bwd_cols_kernel<float><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_cols, s>>>(
+            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+            static_cast<const float*>(dout), stats, static_cast<float*>(dk), static_cast<float*>(dv), nrows, (int)T,
+            (int)D, Wi, c);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swa_backward launch");
     return success();
 }
 

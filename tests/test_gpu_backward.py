@@ -1,0 +1,102 @@
+"""Gradients of the prefill (swa_backward through the C ABI) against the float64 oracle.
+
+Tolerances, from the arithmetic: fp32 operands, every gradient a sum of at most
+2*W products formed and added in fp32 with expf-based weights: 1e-4 absolute on O(1)
+values. bf16 operands (the oracle sees the same bf16 values widened) with bf16 gradients:
+the fp32 results are rounded once to bf16, at most 2^-9 of their magnitude, so the bar is
+4e-3 * max|gradient| + 1e-3."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_causal_b200 as swa
+from sliding_window_causal_b200 import _native, inputs
+from gpu_util import f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def grads_gpu(q, k, v, do, W):
+    out = swa.backward(q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV), W)
+    swa.device_status()
+    return out
+
+
+def check(B, H, T, D, W, dtype, seed):
+    q, k, v = inputs.prefill_inputs(B, H, T, D, dtype, seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    do = torch.randn(B, H, T, D, generator=g).to(dtype)
+    got = grads_gpu(q, k, v, do, W)
+    ref = oracle.backward(f64(q), f64(k), f64(v), f64(do), W)
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        err = float(np.abs(f64(a) - b).max())
+        tol = 1e-4 if dtype == torch.float32 else 4e-3 * float(np.abs(b).max()) + 1e-3
+        assert err <= tol, f"{name}: max err {err} > {tol}"
+
+
+@pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 50, 16, 7), (2, 1, 130, 64, 40), (1, 2, 200, 33, 300),
+                                       (1, 1, 64, 8, 1), (1, 3, 97, 128, 32)])
+def test_backward_fp32(B, H, T, D, W):
+    check(B, H, T, D, W, torch.float32, 11 + T + W)
+
+
+@pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 300, 64, 77), (1, 2, 257, 128, 128), (2, 1, 129, 128, 1000)])
+def test_backward_bf16(B, H, T, D, W):
+    check(B, H, T, D, W, torch.bfloat16, 23 + T + W)
+
+
+def test_backward_mid_size_bf16():
+    """Two heads of a long sequence (T 4096, D 128, W 1024): every element."""
+    check(1, 2, 4096, 128, 1024, torch.bfloat16, 31)
+
+
+def test_backward_matches_gpu_forward_differences():
+    """The gradients give the directional derivative of the GPU fp32 forward itself:
+    sum(dout * (f(x + h u) - f(x - h u))) / 2h against sum(grad * u)."""
+    B, H, T, D, W = 1, 2, 120, 32, 20
+    q, k, v = (t.to(DEV).double().float() for t in inputs.prefill_inputs(B, H, T, D, torch.float32, 41))
+    do = torch.randn(B, H, T, D, device=DEV)
+    grads = swa.backward(q, k, v, do, W)
+    h = 1e-2
+    for which in range(3):
+        u = torch.randn(B, H, T, D, device=DEV)
+        args_p = [q, k, v]
+        args_m = [q, k, v]
+        args_p[which] = args_p[which] + h * u
+        args_m[which] = args_m[which] - h * u
+        fd = float(((swa.forward(*args_p, W) - swa.forward(*args_m, W)) * do).double().sum()) / (2 * h)
+        an = float((grads[which] * u).double().sum())
+        assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), f"operand {which}: {fd} vs {an}"
+    swa.device_status()
+
+
+def test_backward_deterministic():
+    q, k, v = (t.to(DEV) for t in inputs.prefill_inputs(1, 2, 300, 64, torch.bfloat16, 43))
+    do = torch.randn(1, 2, 300, 64, device=DEV).to(torch.bfloat16)
+    a = swa.backward(q, k, v, do, 100)
+    b = swa.backward(q, k, v, do, 100)
+    swa.device_status()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+def test_backward_errors():
+    lib = _native.lib()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    t = torch.zeros(1, 1, 16, 64, device=DEV)
+    need = lib.swa_backward_workspace_bytes(1, 1, 16)
+    assert need == 16 * 8
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    p, w = t.data_ptr(), ws.data_ptr()
+    outs = [torch.empty_like(t).data_ptr() for _ in range(3)]
+    f = lambda *a: lib.swa_backward(p, p, p, p, *outs, *a)
+    assert f(w, need, 1, 1, 16, 64, 4, 0.125, 0, s) == 0
+    assert f(w, need - 8, 1, 1, 16, 64, 4, 0.125, 0, s) == 1     # short workspace
+    assert f(w, need, 1, 1, 16, 64, 0, 0.125, 0, s) == 1         # W < 1
+    assert f(w, need, 1, 1, 16, 64, 4, float("nan"), 0, s) == 1  # scale
+    assert f(None, need, 1, 1, 16, 64, 4, 0.125, 0, s) == 1      # no workspace
+    assert lib.swa_backward_workspace_bytes(-1, 1, 1) == -1
+    swa.device_status()
