@@ -244,7 +244,7 @@ int64_t swa_mha_workspace_bytes(int64_t B, int64_t T, int64_t d_model, int dtype
  *   scale         : the forward's score scale (1/sqrt(D) for swa_forward), finite.
  *   dtype         : SWA_F32 or SWA_BF16; the arithmetic is fp32 on the CUDA cores in both
  *                   cases (bf16 operands are widened, bf16 gradients rounded once).
- *   D             : 1 .. 2048.
+ *   D             : 1 .. 512.
  * The row statistics are recomputed from q and k (no forward state is needed). There are
  * no atomics: the results are deterministic. Errors: as swa_forward_ex, plus a short
  * workspace -> SWA_ERR_INVALID_ARG.

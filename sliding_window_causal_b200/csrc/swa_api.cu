@@ -80,15 +80,12 @@ struct DeviceState {
 };
 std::map<int, DeviceState> g_dev;
 
-constexpr int kBwdMaxD = 2048;
-
 template <typename TIn>
 cudaError_t set_bwd_attrs() {
-    cudaError_t e = cudaFuncSetAttribute(swa::bwd_rows_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         swa::kBwdWarps * (3 * kBwdMaxD + 64) * 4);
+    const int bytes = (int)(swa::bwd_smem_floats(swa::kBwdMaxD) * 4);
+    cudaError_t e = cudaFuncSetAttribute(swa::bwd_rows_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(swa::bwd_cols_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 swa::kBwdWarps * (4 * kBwdMaxD + 64) * 4);
+        e = cudaFuncSetAttribute(swa::bwd_cols_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     return e;
 }
 
@@ -599,7 +596,7 @@ int swa_backward(const void* q, const void* k, const void* v, const void* dout, 
     if (workspace_bytes < swa_backward_workspace_bytes(B, H, T))
         return fail(SWA_ERR_INVALID_ARG, "%s: workspace of %lld bytes, %lld needed", fn, (long long)workspace_bytes,
                     (long long)swa_backward_workspace_bytes(B, H, T));
-    if (D > kBwdMaxD) return fail(SWA_ERR_UNSUPPORTED, "%s: D <= %d", fn, kBwdMaxD);
+    if (D > swa::kBwdMaxD) return fail(SWA_ERR_UNSUPPORTED, "%s: D <= %d", fn, swa::kBwdMaxD);
     const size_t esz = dtype == SWA_BF16 ? 2 : 4;
     const void* ptrs[] = {q, k, v, dout, dq, dk, dv};
     for (const void* p : ptrs)
@@ -607,32 +604,30 @@ int swa_backward(const void* q, const void* k, const void* v, const void* dout, 
     if (!aligned(workspace, 8)) return fail(SWA_ERR_MISALIGNED, "%s: workspace must be 8-byte aligned", fn);
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
-    const int64_t nrows = B * H * T;
-    const int64_t blocks = (nrows + swa::kBwdWarps - 1) / swa::kBwdWarps;
+    const int64_t blocks = B * H * ((T + swa::kBwdRows - 1) / swa::kBwdRows);
     if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
     const int Wi = (int)(W < T ? W : T);
-    const size_t smem_rows = (size_t)swa::kBwdWarps * (3 * D + 64) * 4;
-    const size_t smem_cols = (size_t)swa::kBwdWarps * (4 * D + 64) * 4;
+    const size_t smem = swa::bwd_smem_floats((int)D) * 4;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* stats = static_cast<float*>(workspace);
     const float c = (float)scale;
+    const unsigned grid = (unsigned)blocks, block = swa::kBwdRows * 32;
     if (dtype == SWA_BF16) {
         using T16 = __nv_bfloat16;
-        swa::bwd_rows_kernel<T16><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_rows, s>>>(
+        swa::bwd_rows_kernel<T16><<<grid, block, smem, s>>>(
             static_cast<const T16*>(q), static_cast<const T16*>(k), static_cast<const T16*>(v),
-            static_cast<const T16*>(dout), static_cast<T16*>(dq), stats, nrows, (int)T, (int)D, Wi, c);
-        swa::bwd_cols_kernel<T16><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_cols, s>>>(
+            static_cast<const T16*>(dout), static_cast<T16*>(dq), stats, (int)T, (int)D, Wi, c);
+        swa::bwd_cols_kernel<T16><<<grid, block, smem, s>>>(
             static_cast<const T16*>(q), static_cast<const T16*>(k), static_cast<const T16*>(v),
-            static_cast<const T16*>(dout), stats, static_cast<T16*>(dk), static_cast<T16*>(dv), nrows, (int)T,
-            (int)D, Wi, c);
+            static_cast<const T16*>(dout), stats, static_cast<T16*>(dk), static_cast<T16*>(dv), (int)T, (int)D, Wi, c);
     } else {
-        swa::bwd_rows_kernel<float><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_rows, s>>>(
+        swa::bwd_rows_kernel<float><<<grid, block, smem, s>>>(
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-            static_cast<const float*>(dout), static_cast<float*>(dq), stats, nrows, (int)T, (int)D, Wi, c);
-        swa::bwd_cols_kernel<float><<<(unsigned)blocks, swa::kBwdWarps * 32, smem_cols, s>>>(
+            static_cast<const float*>(dout), static_cast<float*>(dq), stats, (int)T, (int)D, Wi, c);
+        swa::bwd_cols_kernel<float><<<grid, block, smem, s>>>(
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-            static_cast<const float*>(dout), stats, static_cast<float*>(dk), static_cast<float*>(dv), nrows, (int)T,
-            (int)D, Wi, c);
+            static_cast<const float*>(dout), stats, static_cast<float*>(dk), static_cast<float*>(dv), (int)T, (int)D,
+            Wi, c);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "swa_backward launch");

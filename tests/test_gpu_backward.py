@@ -39,7 +39,8 @@ def check(B, H, T, D, W, dtype, seed):
 
 
 @pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 50, 16, 7), (2, 1, 130, 64, 40), (1, 2, 200, 33, 300),
-                                       (1, 1, 64, 8, 1), (1, 3, 97, 128, 32)])
+                                       (1, 1, 64, 8, 1), (1, 3, 97, 128, 32), (1, 1, 45, 300, 9),
+                                       (1, 1, 40, 512, 40)])
 def test_backward_fp32(B, H, T, D, W):
     check(B, H, T, D, W, torch.float32, 11 + T + W)
 
@@ -86,7 +87,7 @@ def test_backward_deterministic():
 def test_backward_errors():
     lib = _native.lib()
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    t = torch.zeros(1, 1, 16, 64, device=DEV)
+    t = torch.zeros(1, 1, 16, 513, device=DEV)
     need = lib.swa_backward_workspace_bytes(1, 1, 16)
     assert need == 16 * 8
     ws = torch.empty(need, dtype=torch.uint8, device=DEV)
@@ -98,5 +99,6 @@ def test_backward_errors():
     assert f(w, need, 1, 1, 16, 64, 0, 0.125, 0, s) == 1         # W < 1
     assert f(w, need, 1, 1, 16, 64, 4, float("nan"), 0, s) == 1  # scale
     assert f(None, need, 1, 1, 16, 64, 4, 0.125, 0, s) == 1      # no workspace
+    assert f(w, need, 1, 1, 16, 513, 4, 0.125, 0, s) == 2        # D above 512
     assert lib.swa_backward_workspace_bytes(-1, 1, 1) == -1
     swa.device_status()
