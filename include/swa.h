@@ -229,32 +229,46 @@ int swa_mha_forward(const void* x, const void* wq, const void* bq, const void* w
 int64_t swa_mha_workspace_bytes(int64_t B, int64_t T, int64_t d_model, int dtype);
 
 /*
+ * swa_forward_lse: swa_forward (contiguous operands, the given scale) that also writes the
+ * natural log-sum-exp of every row's scaled scores, the statistic swa_backward needs:
+ *   lse[b,h,i] = log( sum_{j in band(i)} exp(scale * q_i . k_j) )    [B, H, T] fp32.
+ * Errors: as swa_forward_ex; a null lse -> SWA_ERR_INVALID_ARG.
+ */
+int swa_forward_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, double scale,
+                    int dtype, void* stream);
+
+/*
  * swa_backward: gradients of the prefill with respect to q, k and v.
  *
  * "NNX Sliding-Window Attention" (Mask before softmax) notes that with the band masked to
  * -inf before the softmax the gradients stay well defined. With c = scale and p the
  * forward weights (only band pairs 0 <= i-j < W take part):
  *   dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - delta_i),
- *   delta_i = sum_j p_ij (dout_i . v_j),  dq_i = c sum_j ds_ij k_j,  dk_j = c sum_i ds_ij q_i.
- *   q, k, v, dout : [B,H,T,D] contiguous inputs of `dtype` (dout = dL/dout).
+ *   delta_i = dout_i . out_i,  dq_i = c sum_j ds_ij k_j,  dk_j = c sum_i ds_ij q_i.
+ *   q, k, v       : [B,H,T,D] contiguous inputs of `dtype`.
+ *   out, lse      : the forward's output and log-sum-exp, from swa_forward_lse with the
+ *                   same inputs and scale.
+ *   dout          : [B,H,T,D] = dL/dout, of `dtype`.
  *   dq, dk, dv    : [B,H,T,D] contiguous outputs of `dtype` (overwritten).
  *   workspace     : caller-owned device buffer of workspace_bytes >=
- *                   swa_backward_workspace_bytes(B,H,T) bytes, 8-byte aligned: the per-row
- *                   log-sum-exp and delta the two kernels pass along.
+ *                   swa_backward_workspace_bytes(B,H,T) bytes, 256-byte aligned.
  *   scale         : the forward's score scale (1/sqrt(D) for swa_forward), finite.
- *   dtype         : SWA_F32 or SWA_BF16; the arithmetic is fp32 on the CUDA cores in both
- *                   cases (bf16 operands are widened, bf16 gradients rounded once).
- *   D             : 1 .. 512.
- * The row statistics are recomputed from q and k (no forward state is needed). There are
- * no atomics: the results are deterministic. Errors: as swa_forward_ex, plus a short
- * workspace -> SWA_ERR_INVALID_ARG.
+ *   dtype         : SWA_BF16 with D = 64 or 128 runs on the tensor cores (tcgen05):
+ *                   P and dS are rounded to bf16 for the products, accumulation is fp32,
+ *                   scale must be > 0. Other cases (SWA_F32, or bf16 with another D) run
+ *                   in fp32 on the CUDA cores, D <= 512, recomputing the statistics
+ *                   (out and lse are then not read and may be NULL).
+ * There are no atomics: the results are deterministic. Errors: as swa_forward_ex, plus a
+ * short workspace -> SWA_ERR_INVALID_ARG.
  */
-int swa_backward(const void* q, const void* k, const void* v, const void* dout,
-                 void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
-                 int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, double scale,
-                 int dtype, void* stream);
+int swa_backward(const void* q, const void* k, const void* v, const void* out,
+                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, int64_t workspace_bytes, int64_t B, int64_t H, int64_t T,
+                 int64_t D, int64_t W, double scale, int dtype, void* stream);
 
-/* swa_backward_workspace_bytes: B*H*T*8, or -1 for negative or overflowing sizes. */
+/* swa_backward_workspace_bytes: 8*B*H*Tpad with Tpad = T rounded up to a multiple of 128,
+ * or -1 for negative or overflowing sizes. */
 int64_t swa_backward_workspace_bytes(int64_t B, int64_t H, int64_t T);
 
 /*

@@ -16,7 +16,8 @@ PyTorch only supplies device memory and streams.
     mha_forward(x, wq, bq, wk, bk, wv, bv, wo, bo, num_heads, window)
                                         the multi-head module: projections (cuBLASLt)
                                         around the attention
-    backward(q, k, v, dout, window)     (dq, dk, dv) of the prefill
+    forward_lse(q, k, v, window)        (out, lse): the training forward
+    backward(q, k, v, dout, window)     (dq, dk, dv) of the prefill (tensor cores for bf16)
     forward_host(...)                   prefill from pinned host tensors (copies included)
 """
 import ctypes
@@ -24,7 +25,7 @@ import ctypes
 from . import _native
 from ._native import SWA_BF16, SWA_F32, SwaError, check
 
-__all__ = ["forward", "backward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
+__all__ = ["forward", "forward_lse", "backward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
            "mha_workspace_bytes", "forward_host", "device_status", "tile_class", "valid_slots",
            "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
 
@@ -105,10 +106,29 @@ def forward(q, k, v, window, out=None, scale=None):
     return out.squeeze(1) if squeeze else out
 
 
-def backward(q, k, v, dout, window, scale=None):
+def forward_lse(q, k, v, window, scale=None):
+    """Training forward: (out, lse) for contiguous [B,H,T,D] q, k, v; lse [B,H,T] fp32 is
+    the natural log-sum-exp of each row's scaled scores (what backward needs)."""
+    torch = _torch()
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B,H,T,D] shape")
+    dev = _need_cuda(q, k, v)
+    B, H, T, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    sc = 1.0 / D ** 0.5 if scale is None else float(scale)
+    with torch.cuda.device(dev):
+        check(_native.lib().swa_forward_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                            lse.data_ptr(), B, H, T, D, int(window), sc, _dtype_code(q),
+                                            _stream_ptr(dev)))
+    return out, lse
+
+
+def backward(q, k, v, dout, window, scale=None, out=None, lse=None):
     """Gradients (dq, dk, dv) of the prefill output with respect to q, k, v, given the
-    output gradient dout. All [B,H,T,D] contiguous CUDA tensors of one dtype (fp32 or
-    bf16, D <= 2048); fp32 arithmetic on the CUDA cores. scale defaults to 1/sqrt(D)."""
+    output gradient dout. All [B,H,T,D] contiguous CUDA tensors of one dtype. out and lse
+    are the forward's (forward_lse); they are computed here when not given. bf16 with D
+    64 or 128 runs on the tensor cores; other cases on the CUDA cores (D <= 512)."""
     torch = _torch()
     if q.dim() != 4 or any(t.shape != q.shape for t in (k, v, dout)):
         raise ValueError("q, k, v, dout must share one [B,H,T,D] shape")
@@ -116,14 +136,18 @@ def backward(q, k, v, dout, window, scale=None):
         raise TypeError("q, k, v, dout must share one dtype")
     dev = _need_cuda(q, k, v, dout)
     B, H, T, D = q.shape
+    tensor_cores = q.dtype == torch.bfloat16 and D in (64, 128)
+    if tensor_cores and (out is None or lse is None):
+        out, lse = forward_lse(q, k, v, window, scale)
+    ptr = lambda t: None if t is None else t.data_ptr()
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     lib = _native.lib()
     ws = torch.empty(max(1, int(lib.swa_backward_workspace_bytes(B, H, T))), dtype=torch.uint8, device=dev)
     sc = 1.0 / D ** 0.5 if scale is None else float(scale)
     with torch.cuda.device(dev):
-        check(lib.swa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
-                               dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, H, T, D,
-                               int(window), sc, _dtype_code(q), _stream_ptr(dev)))
+        check(lib.swa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ptr(out), dout.data_ptr(),
+                               ptr(lse), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                               ws.numel(), B, H, T, D, int(window), sc, _dtype_code(q), _stream_ptr(dev)))
     return dq, dk, dv
 
 

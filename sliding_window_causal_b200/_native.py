@@ -12,7 +12,7 @@ LIB_PATH = os.path.join(_HERE, "_swa.so")
 # every exported symbol of include/swa.h
 EXPORTS = ("swa_forward", "swa_forward_ex", "swa_band_weights", "swa_decode", "swa_decode_noalloc",
            "swa_chunk_forward", "swa_ring_append", "swa_mha_forward", "swa_mha_workspace_bytes",
-           "swa_backward", "swa_backward_workspace_bytes", "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
+           "swa_forward_lse", "swa_backward", "swa_backward_workspace_bytes", "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
            "swa_set_wait_limit_ns", "swa_timeout_probe")
 
 SWA_F32, SWA_BF16 = 0, 1
@@ -57,7 +57,9 @@ def lib(path=None):
     h.swa_mha_forward.restype = i32
     h.swa_mha_workspace_bytes.argtypes = [i64, i64, i64, i32]
     h.swa_mha_workspace_bytes.restype = i64
-    h.swa_backward.argtypes = [vp] * 8 + [i64] * 6 + [ctypes.c_double, i32, vp]
+    h.swa_forward_lse.argtypes = [vp] * 5 + [i64] * 5 + [ctypes.c_double, i32, vp]
+    h.swa_forward_lse.restype = i32
+    h.swa_backward.argtypes = [vp] * 10 + [i64] * 6 + [ctypes.c_double, i32, vp]
     h.swa_backward.restype = i32
     h.swa_backward_workspace_bytes.argtypes = [i64, i64, i64]
     h.swa_backward_workspace_bytes.restype = i64

@@ -1,0 +1,435 @@
+// backward_tc.cuh: gradients of the bf16 sliding-window prefill on the sm_100a tensor
+// cores (D = 64 or 128).
+//
+// The gradients ("NNX Sliding-Window Attention", Mask before softmax: well defined for
+// finite allowed scores), with s_ij = q_i . k_j, c the scale, P_ij = exp(c s_ij - lse_i)
+// the forward weights and delta_i = dout_i . out_i:
+//   dV = P^T dO,   dS = P o (dO V^T - delta),   dK = c dS^T Q,   dQ = c dS K
+// over the band pairs only. Three kernels, no atomics (deterministic):
+//   bwd_stats_kernel  delta_i from dout and out, and lse_i (from the forward) in log2
+//                     units, into a [B*H, Tpad] layout padded to whole 128-row tiles
+//                     (padding rows get lse = +inf, delta = 0, so they weigh nothing).
+//   bwd_kv_kernel<D>  one CTA per (b, h, 128-key tile): K and V stay in shared memory;
+//                     for every query tile that meets the band, TMA brings Q, dO and the
+//                     tile's (lse, delta); S^T = K Q^T and dP^T = V dO^T go to TMEM; four
+//                     warps (one key row each) turn them into bf16 P^T and dS^T over the
+//                     same TMEM columns; then dV += P^T dO and dK += dS^T Q accumulate in
+//                     TMEM (TS form: A from TMEM, B from shared memory).
+//   bwd_q_kernel<D>   one CTA per (b, h, 128-query tile): Q and dO stay; for every key
+//                     tile of the band S = Q K^T and dP = dO V^T, then dS (bf16, in TMEM)
+//                     and dQ += dS K.
+// Work per band pair: seven 128x128xD products (the score and dP products are formed in
+// both kernels, so that neither needs atomics), against five in the useful-FLOP count.
+// Every mbarrier wait is bounded as in the forward kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "plan.h"
+#include "prefill_pp.cuh"
+#include "ptx.cuh"
+#include "umma.h"
+
+namespace swa {
+
+constexpr int kBwdTcThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 element-wise
+
+template <int D>
+struct BwdTcCfg {
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static constexpr int kBoxBytes = 128 * 128;
+    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kStages = D == 128 ? 4 : 8;  // streamed tiles (Q/dO or K/V)
+    static constexpr int kFixOff = 0;                 // two resident tiles
+    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kStatStages = 2;
+    static constexpr int kStatBytes = 2 * 128 * 4;    // lse2[128], delta[128]
+    static constexpr int kStatOff = kRingOff + kStages * kTileBytes;
+    static constexpr int kBarOff = kStatOff + kStatStages * kStatBytes;
+    // fix_full, ring_full[S], ring_empty[S], stat_full[2], stat_empty[2], s_full, p_full,
+    // o_final, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 384;
+};
+
+// delta_i = sum_d dout_i[d] out_i[d] (fp32) and lse2_i = lse_i * log2(e), one warp per row.
+__global__ void __launch_bounds__(256)
+    bwd_stats_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
+                     const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
+                     int64_t BH, int T, int Tpad, int D) {
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= BH * Tpad) return;
+    const int64_t bh = r / Tpad;
+    const int i = (int)(r - bh * Tpad);
+    if (i >= T) {
+        if (lane == 0) {
+            lse2[r] = INFINITY;
+            delta[r] = 0.f;
+        }
+        return;
+    }
+    const int64_t src = (bh * T + i) * D;
+    float acc = 0.f;
+    for (int d = lane; d < D; d += 32)
+        acc = fmaf(__bfloat162float(dout[src + d]), __bfloat162float(out[src + d]), acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+        delta[r] = acc;
+        lse2[r] = lse[bh * T + i] * 1.4426950408889634f;
+    }
+}
+
+// One chunk of 32 columns of one TMEM row: scores s (fp32, raw q.k) and dp, to bf16 P and
+// dS = P (dp - delta): P = exp2(s*c2 - lse2) where the column is valid, else 0. Column
+// t's lse2 and delta come from lse2_of(t), delta_of(t); valid_of(t) masks edge tiles.
+template <bool STORE_P, typename Lse, typename Delta, typename Valid>
+__device__ __forceinline__ void bwd_chunk(uint32_t scol, uint32_t dpcol, float c2, Lse lse2_of, Delta delta_of,
+                                          Valid valid_of) {
+    uint32_t s[32], dp[32];
+    ptx::tmem_ld32(scol, s);
+    ptx::tmem_ld32(dpcol, dp);
+    ptx::tmem_ld_wait();
+    ptx::reg_fence(s);
+    ptx::reg_fence(dp);
+    uint32_t ph[16], dh[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        float p[2], ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int col = 2 * t + e;
+            const float pe = valid_of(col) ? ptx::ex2(__uint_as_float(s[col]) * c2 - lse2_of(col)) : 0.f;
+            p[e] = pe;
+            ds[e] = pe * (__uint_as_float(dp[col]) - delta_of(col));
+        }
+        ph[t] = ptx::pack_bf16x2(p[0], p[1]);
+        dh[t] = ptx::pack_bf16x2(ds[0], ds[1]);
+    }
+    if (STORE_P) ptx::tmem_st16(scol, ph);
+    ptx::tmem_st16(STORE_P ? dpcol : scol, dh);
+}
+
+// Store one 128-column TMEM accumulator row (D fp32 values from column col) times a, as
+// bf16, to dst (a row of D elements), 16 bytes at a time.
+template <int D>
+__device__ __forceinline__ void bwd_store_row(uint32_t col, float a, __nv_bfloat16* dst, bool live) {
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld32(col + cc * 32, o);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(o);
+        if (live) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                uint4 val;
+                val.x = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 0]) * a, __uint_as_float(o[8 * t + 1]) * a);
+                val.y = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 2]) * a, __uint_as_float(o[8 * t + 3]) * a);
+                val.z = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 4]) * a, __uint_as_float(o[8 * t + 5]) * a);
+                val.w = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 6]) * a, __uint_as_float(o[8 * t + 7]) * a);
+                *reinterpret_cast<uint4*>(dst + cc * 32 + t * 8) = val;
+            }
+        }
+    }
+}
+
+// KV = true: bwd_kv_kernel (resident K, V; streamed Q, dO; dK, dV out).
+// KV = false: bwd_q_kernel (resident Q, dO; streamed K, V; dQ out).
+// Maps are 4-D {D, T, H, B} of contiguous [B,H,T,D] tensors. lse2/delta: [B*H, Tpad].
+template <int D, bool KV>
+__global__ void __launch_bounds__(kBwdTcThreads, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const float* __restrict__ lse2, const float* __restrict__ delta, __nv_bfloat16* __restrict__ g1,
+                  __nv_bfloat16* __restrict__ g2, int H, int T, int Tpad, int W, int n_t, float c, float c2,
+                  uint64_t wait_limit_ns, int* status) {
+    using Cf = BwdTcCfg<D>;
+    constexpr int NS = Cf::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
+    uint64_t* fix_full = bars;
+    uint64_t* ring_full = bars + 1;  // [NS]
+    uint64_t* ring_empty = ring_full + NS;
+    uint64_t* stat_full = ring_empty + NS;  // [2]
+    uint64_t* stat_empty = stat_full + 2;   // [2]
+    uint64_t* s_full = stat_empty + 2;
+    uint64_t* p_full = s_full + 1;
+    uint64_t* o_final = p_full + 1;
+    uint64_t* drain = o_final + 1;
+    const float* st_smem = reinterpret_cast<const float*>(smem + Cf::kStatOff);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cf::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x / n_t;
+    const int xt = blockIdx.x - bh * n_t;  // the resident tile: key tile (KV) or query tile
+    const int b = bh / H, h = bh - b * H;
+    // the streamed tiles that meet the band: query tiles xt .. (KV), or key tiles (Q)
+    int lo, hi;
+    if (KV) {
+        lo = xt;
+        hi = min(n_t - 1, (128 * xt + 127 + W - 1) / 128);
+    } else {
+        int64_t f, l;
+        kv_tile_range(T, W, 128, 128, xt, &f, &l);
+        lo = (int)f;
+        hi = (int)l;
+    }
+    auto cls = [&](int yt) { return KV ? tile_class(T, W, 128, 128, yt, xt) : tile_class(T, W, 128, 128, xt, yt); };
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(fix_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(ring_full + s, 1);
+            ptx::mbar_init(ring_empty + s, 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            ptx::mbar_init(stat_full + x, 1);
+            ptx::mbar_init(stat_empty + x, 128);
+        }
+        ptx::mbar_init(s_full, 1);
+        ptx::mbar_init(p_full, 128);
+        ptx::mbar_init(o_final, 1);
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
+        ptx::prefetch_tmap(&tm_do);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, Cf::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t loads = 0, stat_loads = 0;
+    bool fix_issued = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- producer
+            bool ok = true;
+            const CUtensorMap* fa = KV ? &tm_k : &tm_q;   // resident operands
+            const CUtensorMap* fb = KV ? &tm_v : &tm_do;
+            const CUtensorMap* sa = KV ? &tm_q : &tm_k;   // streamed operands
+            const CUtensorMap* sb = KV ? &tm_do : &tm_v;
+            ptx::mbar_arrive_expect_tx(fix_full, 2 * Cf::kTileBytes);
+            for (int x = 0; x < 2; ++x)
+                for (int cc = 0; cc < D / 64; ++cc)
+                    ptx::tma_load_4d(smem + Cf::kFixOff + x * Cf::kTileBytes + cc * Cf::kBoxBytes, x ? fb : fa,
+                                     fix_full, cc * 64, 128 * xt, h, b);
+            fix_issued = true;
+            for (int yt = lo; yt <= hi && ok; ++yt) {
+                if (cls(yt) == 0) continue;
+                for (int x = 0; x < 2 && ok; ++x) {
+                    const uint32_t st = loads % NS;
+                    if (loads >= (uint32_t)NS)
+                        ok = ptx::mbar_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag);
+                    if (!ok) break;
+                    uint8_t* dst = smem + Cf::kRingOff + st * Cf::kTileBytes;
+                    ptx::mbar_arrive_expect_tx(ring_full + st, Cf::kTileBytes);
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        ptx::tma_load_4d(dst + cc * Cf::kBoxBytes, x ? sb : sa, ring_full + st, cc * 64, 128 * yt, h, b);
+                    ++loads;
+                }
+                if (KV && ok) {
+                    // the query tile's lse2 and delta (512 bytes each, contiguous in [B*H, Tpad])
+                    const uint32_t ss = stat_loads % 2;
+                    if (stat_loads >= 2)
+                        ok = ptx::mbar_wait(stat_empty + ss, ((stat_loads / 2) - 1) & 1, wait_limit_ns, abort_flag);
+                    if (!ok) break;
+                    uint8_t* dst = smem + Cf::kStatOff + ss * Cf::kStatBytes;
+                    ptx::mbar_arrive_expect_tx(stat_full + ss, Cf::kStatBytes);
+                    const int64_t off = (int64_t)bh * Tpad + 128 * yt;
+                    ptx::bulk_load(dst, lse2 + off, 512, stat_full + ss);
+                    ptx::bulk_load(dst + 512, delta + off, 512, stat_full + ss);
+                    ++stat_loads;
+                }
+            }
+            if (!ok) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
+            const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
+            const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
+            const uint32_t lo_k = (uint32_t)umma::smem_desc(0, 16, 1024);
+            const uint32_t lo_mn = (uint32_t)umma::smem_desc(0, Cf::kBoxBytes, 1024);
+            const uint32_t fa_lo = ptx::smem_u32(smem + Cf::kFixOff) >> 4;
+            const uint32_t fb_lo = ptx::smem_u32(smem + Cf::kFixOff + Cf::kTileBytes) >> 4;
+            const uint32_t ring_lo = ptx::smem_u32(smem + Cf::kRingOff) >> 4;
+            constexpr uint32_t kStageLo = Cf::kTileBytes >> 4;
+            bool ok = ptx::mbar_wait(fix_full, 0, wait_limit_ns, abort_flag);
+            uint32_t L = 0;
+            int j = 0;  // visited tiles
+            for (int yt = lo; yt <= hi && ok; ++yt) {
+                if (cls(yt) == 0) continue;
+                const uint32_t sta = L % NS, stb = (L + 1) % NS;
+                ok = ptx::mbar_wait(ring_full + sta, (L / NS) & 1, wait_limit_ns, abort_flag);
+                if (ok) ok = ptx::mbar_wait(ring_full + stb, ((L + 1) / NS) & 1, wait_limit_ns, abort_flag);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a_lo = ring_lo + sta * kStageLo, b_lo = ring_lo + stb * kStageLo;
+                // KV: S^T = K Q^T, dP^T = V dO^T.   Q: S = Q K^T, dP = dO V^T.
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k), desc_hi | ((a_lo + off) | lo_k),
+                                idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + Cf::kColDP, desc_hi | ((fb_lo + off) | lo_k), desc_hi | ((b_lo + off) | lo_k),
+                                idesc_s, kk > 0 ? 1u : 0u);
+                }
+                ptx::tc_commit(s_full);
+                ok = ptx::mbar_wait(p_full, j & 1, wait_limit_ns, abort_flag);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (KV) {
+                    // dV += P^T dO (B = dO, the streamed b tile); dK += dS^T Q (B = Q, the streamed a tile)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColS + pp_pcol(kk),
+                                    desc_hi | ((b_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ts(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
+                                    desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    // dQ += dS K (A = dS over the S columns, B = K, the streamed a tile)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColS + pp_pcol(kk),
+                                    desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::tc_commit(ring_empty + sta);
+                ptx::tc_commit(ring_empty + stb);
+                L += 2;
+                ++j;
+            }
+            if (ok) ptx::tc_commit(o_final);
+            if (!ok) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        // -------------------------------------------------------------------- element-wise
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;  // the TMEM lane = this thread's resident row
+        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+        const int xr = 128 * xt + r;         // key index (KV) or query index (Q)
+        float my_lse2 = 0.f, my_delta = 0.f;
+        if (!KV) {
+            my_lse2 = lse2[(int64_t)bh * Tpad + xr];  // +inf on padding rows: P = 0
+            my_delta = delta[(int64_t)bh * Tpad + xr];
+        }
+        bool ok = true;
+        int j = 0;
+        for (int yt = lo; yt <= hi && ok; ++yt) {
+            const int k = cls(yt);
+            if (k == 0) continue;
+            bool w = ptx::mbar_wait(s_full, j & 1, wait_limit_ns, abort_flag);
+            const float* sts = st_smem + (j & 1) * 256;
+            if (KV && w) w = ptx::mbar_wait(stat_full + (j & 1), (j >> 1) & 1, wait_limit_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const bool edge = k != 2;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                const int y0 = 128 * yt + 32 * cc;  // index of this chunk's first column
+                if (KV) {
+                    // row = key j = xr, columns = queries i = y0 + t: valid iff 0 <= i - j < W, i < T
+                    auto lse_of = [&](int t) { return sts[32 * cc + t]; };
+                    auto delta_of = [&](int t) { return sts[128 + 32 * cc + t]; };
+                    auto valid = [&](int t) {
+                        const int d = y0 + t - xr;
+                        return !edge || (d >= 0 && d < W && y0 + t < T && xr < T);
+                    };
+                    bwd_chunk<true>(tl + Cf::kColS + 32 * cc, tl + Cf::kColDP + 32 * cc, c2, lse_of, delta_of, valid);
+                } else {
+                    // row = query i = xr, columns = keys j = y0 + t
+                    auto lse_of = [&](int) { return my_lse2; };
+                    auto delta_of = [&](int) { return my_delta; };
+                    auto valid = [&](int t) {
+                        const int d = xr - (y0 + t);
+                        return !edge || (d >= 0 && d < W && y0 + t < T && xr < T);
+                    };
+                    bwd_chunk<false>(tl + Cf::kColS + 32 * cc, tl + Cf::kColDP + 32 * cc, c2, lse_of, delta_of, valid);
+                }
+            }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            if (KV) ptx::mbar_arrive(stat_empty + (j & 1));
+            ptx::mbar_arrive(p_full);
+            ++j;
+        }
+        if (ok) {
+            const bool w = ptx::mbar_wait(o_final, 0, wait_limit_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, w)) ok = false;
+        }
+        if (ok) {
+            ptx::tc_fence_after();
+            const bool live = xr < T;
+            const int64_t row = ((int64_t)bh * T + xr) * D;
+            if (KV) {
+                bwd_store_row<D>(tl + Cf::kColB, c, g1 + row, live);    // dK = c dS^T Q
+                bwd_store_row<D>(tl + Cf::kColA, 1.f, g2 + row, live);  // dV = P^T dO
+            } else {
+                bwd_store_row<D>(tl + Cf::kColA, c, g1 + row, live);    // dQ = c dS K
+            }
+        } else {
+            atomicCAS(status, 0, 5);
+            *abort_flag = 1;
+        }
+    }
+
+    // -------------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        if (warp == 0 && lane == 0) {
+            if (fix_issued) ptx::mbar_wait(fix_full, 0, kPPDrainLimitNs, nullptr);
+            for (uint32_t st = 0; st < (uint32_t)NS && st < loads; ++st) {
+                const uint32_t t = st + ((loads - 1 - st) / NS) * NS;
+                ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);
+            }
+            for (uint32_t ss = 0; ss < 2 && ss < stat_loads; ++ss) {
+                const uint32_t t = ss + ((stat_loads - 1 - ss) / 2) * 2;
+                ptx::mbar_wait(stat_full + ss, (t / 2) & 1, kPPDrainLimitNs, nullptr);
+            }
+        }
+        if (warp == 1 && lane == 0) {
+            ptx::tc_commit(drain);
+            ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cf::kTmemCols);
+    }
+}
+
+}  // namespace swa

@@ -204,16 +204,19 @@ __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scal
                     v[c][t] = __float_as_uint(-INFINITY);
             }
     }
-    float q[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    // eight independent max chains, so that the row maximum is not one long dependent chain
+    float q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int t = 0; t < 32; t += 8) {
+        for (int t = 0; t < 32; t += 16) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 8; ++j)
                 q[j] = ptx::max3(q[j], __uint_as_float(v[c][t + 2 * j]), __uint_as_float(v[c][t + 2 * j + 1]));
         }
-    const float tm = fmaxf(fmaxf(q[0], q[1]), fmaxf(q[2], q[3])) * scale_log2;
+    const float tm = ptx::max3(ptx::max3(q[0], q[1], q[2]), ptx::max3(q[3], q[4], q[5]), fmaxf(q[6], q[7])) * scale_log2;
     const bool need = m != -INFINITY && tm > m + kPPRescaleThreshold;
     if (__any_sync(0xffffffffu, need)) {
         const int k = need ? min(126, (int)ceilf(tm - m)) : 0;
@@ -250,12 +253,14 @@ __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scal
     l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
-template <int D>
+// LSE: also write the natural log-sum-exp of each row (a separate instantiation, so that
+// the plain prefill keeps its register allocation).
+template <int D, bool LSE = false>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-                      int64_t osb, int64_t osh, int64_t ost, int BH, int H, int T, int W, int n_qt,
-                      float scale_log2, uint64_t wait_limit_ns,
+                      int64_t osb, int64_t osh, int64_t ost, float* __restrict__ lse, int BH, int H,
+                      int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
                       int* status) {
     using C = PPCfg<D>;
     constexpr int NS = C::kStages;
@@ -504,6 +509,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             ptx::tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            // natural log-sum-exp of the row's scaled scores: (m + log2 l) ln 2
+            if (LSE && i < T) lse[((int64_t)it.b * H + it.h) * T + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
             __nv_bfloat16* orow = out + it.b * osb + it.h * osh + (int64_t)i * ost;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {

@@ -37,7 +37,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 __global__ void __launch_bounds__(kSimtWarps * 32)
     prefill_simt_kernel(const float* __restrict__ q, const float* __restrict__ k,
                         const float* __restrict__ v, float* __restrict__ out, Strides st,
-                        int64_t nrows, int H, int T, int D, int W, float scale) {
+                        float* __restrict__ lse, int64_t nrows, int H, int T, int D, int W, float scale) {
     extern __shared__ float sm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kSimtWarps + warp;
@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
     }
     float* orow = out + b * st.o[0] + h * st.o[1] + (int64_t)i * st.o[2];
     for (int d = lane; d < D; d += 32) orow[d] = sacc[d] / l;
+    if (lse != nullptr && lane == 0) lse[r] = m + logf(l);  // natural log-sum-exp
 }
 
 }  // namespace swa

@@ -17,6 +17,7 @@
 #include "swa.h"
 #include "api_internal.h"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "chunk.cuh"
 #include "decode.cuh"
 #include "plan.h"
@@ -80,6 +81,16 @@ struct DeviceState {
 };
 std::map<int, DeviceState> g_dev;
 
+template <int D>
+cudaError_t set_bwd_tc_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(swa::bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         swa::BwdTcCfg<D>::kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(swa::bwd_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 swa::BwdTcCfg<D>::kSmemBytes);
+    return e;
+}
+
 template <typename TIn>
 cudaError_t set_bwd_attrs() {
     const int bytes = (int)(swa::bwd_smem_floats(swa::kBwdMaxD) * 4);
@@ -112,6 +123,16 @@ int device_state(DeviceState** out) {
             e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::PPCfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<128, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::PPCfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::PPCfg<64>::kSmemBytes);
+        if (e == cudaSuccess) e = set_bwd_tc_attrs<64>();
+        if (e == cudaSuccess) e = set_bwd_tc_attrs<128>();
         if (e == cudaSuccess) e = set_bwd_attrs<float>();
         if (e == cudaSuccess) e = set_bwd_attrs<__nv_bfloat16>();
         if (e == cudaSuccess)
@@ -124,11 +145,14 @@ int device_state(DeviceState** out) {
             e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e == cudaSuccess) {
             // The register split inside the kernel assumes this launch allocation.
-            cudaFuncAttributes a128, a64;
+            cudaFuncAttributes a128, a64, l128, l64;
             e = cudaFuncGetAttributes(&a128, swa::prefill_pp_kernel<128>);
             if (e == cudaSuccess) e = cudaFuncGetAttributes(&a64, swa::prefill_pp_kernel<64>);
+            if (e == cudaSuccess) e = cudaFuncGetAttributes(&l128, swa::prefill_pp_kernel<128, true>);
+            if (e == cudaSuccess) e = cudaFuncGetAttributes(&l64, swa::prefill_pp_kernel<64, true>);
             st.pp_regs_ok = e == cudaSuccess && a128.numRegs == swa::kPPLaunchRegs &&
-                            a64.numRegs == swa::kPPLaunchRegs;
+                            a64.numRegs == swa::kPPLaunchRegs && l128.numRegs == swa::kPPLaunchRegs &&
+                            l64.numRegs == swa::kPPLaunchRegs;
         }
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::prefill_simt_kernel,
@@ -290,7 +314,7 @@ int check_sizes(const char* fn, int64_t B, int64_t H, int64_t T, int64_t D, int6
 
 int forward_impl(const char* fn, const void* q, const void* k, const void* v, void* out, int64_t B,
                  int64_t H, int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides,
-                 int dtype, void* stream) {
+                 int dtype, void* stream, float* lse = nullptr) {
     if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
     if (B == 0 || H == 0 || T == 0) return success();
     if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
@@ -332,13 +356,21 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
         const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
         const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
         auto* ob = static_cast<__nv_bfloat16*>(out);
-        if (D == 128)
+        if (D == 128 && lse)
+            swa::prefill_pp_kernel<128, true><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
+                scale_log2, wait_limit(), ds->status);
+        else if (D == 128)
             swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], (int)BH, (int)H, (int)T, Wi, n_qt,
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
+                scale_log2, wait_limit(), ds->status);
+        else if (lse)
+            swa::prefill_pp_kernel<64, true><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
                 scale_log2, wait_limit(), ds->status);
         else
             swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], (int)BH, (int)H, (int)T, Wi, n_qt,
+                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
                 scale_log2, wait_limit(), ds->status);
     } else {
         if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: fp32 supports D <= 4096", fn);
@@ -357,7 +389,7 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
         }
         swa::prefill_simt_kernel<<<(unsigned)blocks, swa::kSimtWarps * 32, smem, s>>>(
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-            static_cast<float*>(out), sx, nrows, (int)H, (int)T, (int)D, Wi, (float)scale);
+            static_cast<float*>(out), sx, lse, nrows, (int)H, (int)T, (int)D, Wi, (float)scale);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "swa_forward launch");
@@ -581,21 +613,81 @@ int swa_chunk_forward(const void* q, const void* k, const void* v, void* kring, 
 
 int64_t swa_backward_workspace_bytes(int64_t B, int64_t H, int64_t T) {
     if (B < 0 || H < 0 || T < 0) return -1;
-    if (B > 0 && H > 0 && T > 0 && (B * H > INT64_MAX / T || B * H * T > INT64_MAX / 8)) return -1;
-    return B * H * T * 8;
+    const int64_t Tpad = (T + 127) / 128 * 128;
+    if (B > 0 && H > 0 && Tpad > 0 && (B * H > INT64_MAX / Tpad || B * H * Tpad > INT64_MAX / 8)) return -1;
+    return B * H * Tpad * 8;
 }
 
-int swa_backward(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
-                 void* workspace, int64_t workspace_bytes, int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
-                 double scale, int dtype, void* stream) {
+int swa_forward_lse(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t H,
+                    int64_t T, int64_t D, int64_t W, double scale, int dtype, void* stream) {
+    if (!lse && B > 0 && H > 0 && T > 0) return fail(SWA_ERR_INVALID_ARG, "swa_forward_lse: null lse");
+    if (lse && !aligned(lse, 4)) return fail(SWA_ERR_MISALIGNED, "swa_forward_lse: lse must be 4-byte aligned");
+    return forward_impl("swa_forward_lse", q, k, v, out, B, H, T, D, W, scale, nullptr, dtype, stream, lse);
+}
+
+int swa_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+                 int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, double scale, int dtype, void* stream) {
     const char* fn = "swa_backward";
     if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
     if (B == 0 || H == 0 || T == 0) return success();
-    if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace)
+    const bool tc = dtype == SWA_BF16 && (D == 64 || D == 128);
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace || (tc && (!out || !lse)))
         return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
     if (workspace_bytes < swa_backward_workspace_bytes(B, H, T))
         return fail(SWA_ERR_INVALID_ARG, "%s: workspace of %lld bytes, %lld needed", fn, (long long)workspace_bytes,
                     (long long)swa_backward_workspace_bytes(B, H, T));
+    if (tc) {
+        const void* ptrs16[] = {q, k, v, out, dout, dq, dk, dv};
+        for (const void* p : ptrs16)
+            if (!aligned(p, 16)) return fail(SWA_ERR_MISALIGNED, "%s: bf16 tensors must be 16-byte aligned", fn);
+        if (!aligned(workspace, 256) || !aligned(lse, 4))
+            return fail(SWA_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned, lse 4-byte", fn);
+        if (!(scale > 0.0)) return fail(SWA_ERR_UNSUPPORTED, "%s: the bf16 path needs scale > 0", fn);
+        DeviceState* ds;
+        if (int rc = device_state(&ds)) return rc;
+        const int64_t BH = B * H;
+        const int n_t = (int)((T + 127) / 128);
+        const int64_t Tpad = (int64_t)n_t * 128;
+        if (BH * n_t > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+        const int64_t cst[3] = {H * T * D, T * D, D};
+        CUtensorMap mq, mk, mv, mdo;
+        int rc;
+        if ((rc = make_map(&mq, q, B, H, T, D, cst)) || (rc = make_map(&mk, k, B, H, T, D, cst)) ||
+            (rc = make_map(&mv, v, B, H, T, D, cst)) || (rc = make_map(&mdo, dout, B, H, T, D, cst)))
+            return rc;
+        cudaStream_t s = static_cast<cudaStream_t>(stream);
+        float* lse2 = static_cast<float*>(workspace);
+        float* delta = lse2 + BH * Tpad;
+        const int Wi = (int)(W < T ? W : T);
+        swa::bwd_stats_kernel<<<(unsigned)((BH * Tpad + 7) / 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), lse, lse2, delta, BH,
+            (int)T, (int)Tpad, (int)D);
+        const float c = (float)scale, c2 = (float)(1.4426950408889634 * scale);
+        const unsigned grid = (unsigned)(BH * n_t);
+        auto* gq = static_cast<__nv_bfloat16*>(dq);
+        auto* gk = static_cast<__nv_bfloat16*>(dk);
+        auto* gv = static_cast<__nv_bfloat16*>(dv);
+        if (D == 128) {
+            swa::bwd_tc_kernel<128, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, lse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                ds->status);
+            swa::bwd_tc_kernel<128, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, lse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                ds->status);
+        } else {
+            swa::bwd_tc_kernel<64, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, lse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                ds->status);
+            swa::bwd_tc_kernel<64, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, lse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                ds->status);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "swa_backward launch");
+        return success();
+    }
+    // CUDA-core path: the row statistics are recomputed from q and k
     if (D > swa::kBwdMaxD) return fail(SWA_ERR_UNSUPPORTED, "%s: D <= %d", fn, swa::kBwdMaxD);
     const size_t esz = dtype == SWA_BF16 ? 2 : 4;
     const void* ptrs[] = {q, k, v, dout, dq, dk, dv};

@@ -112,3 +112,19 @@ def test_split_plan_covers_window():
         assert (S - 1) * chunk < W <= S * chunk
     with pytest.raises(swa.SwaError):
         swa.split_plan(1, 1, 96, 10)
+
+
+def test_workspace_sizes():
+    """The workspace queries (host only): the backward's rows are padded to whole 128-row
+    tiles, two fp32 values each; the module's four [B*T, d] parts are rounded up to 256
+    bytes, plus 32 MiB of GEMM scratch. Invalid sizes give -1."""
+    lib = _native.lib()
+    for (B, H, T) in ((1, 1, 1), (2, 3, 128), (1, 32, 16384), (4, 2, 129), (0, 5, 7)):
+        tpad = (T + 127) // 128 * 128
+        assert lib.swa_backward_workspace_bytes(B, H, T) == 8 * B * H * tpad
+    assert lib.swa_backward_workspace_bytes(-1, 1, 1) == -1
+    for (B, T, d, dt, esz) in ((1, 5, 2, 0, 4), (1, 16384, 4096, 1, 2), (2, 300, 256, 1, 2)):
+        part = (B * T * d * esz + 255) // 256 * 256
+        assert lib.swa_mha_workspace_bytes(B, T, d, dt) == 4 * part + (32 << 20)
+    assert lib.swa_mha_workspace_bytes(1, 5, 0, 1) == -1
+    assert lib.swa_mha_workspace_bytes(1, 5, 8, 7) == -1

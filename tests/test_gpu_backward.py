@@ -1,10 +1,11 @@
 """Gradients of the prefill (swa_backward through the C ABI) against the float64 oracle.
 
-Tolerances, from the arithmetic: fp32 operands, every gradient a sum of at most
-2*W products formed and added in fp32 with expf-based weights: 1e-4 absolute on O(1)
-values. bf16 operands (the oracle sees the same bf16 values widened) with bf16 gradients:
-the fp32 results are rounded once to bf16, at most 2^-9 of their magnitude, so the bar is
-4e-3 * max|gradient| + 1e-3."""
+Tolerances, from the arithmetic: fp32 operands (CUDA cores), every gradient a sum of at
+most 2*W products formed and added in fp32 with expf-based weights: 1e-4 absolute on O(1)
+values. bf16 operands (the oracle sees the same bf16 values widened): on the tensor cores
+P and dS are rounded to bf16 before their products, the forward output that delta is
+formed from is bf16, and each gradient is rounded once to bf16; each rounding is at most
+2^-9 relative and unbiased, so the bar is 1e-2 * max|gradient| + 2e-3."""
 import ctypes
 
 import numpy as np
@@ -34,7 +35,7 @@ def check(B, H, T, D, W, dtype, seed):
     ref = oracle.backward(f64(q), f64(k), f64(v), f64(do), W)
     for name, a, b in zip(("dq", "dk", "dv"), got, ref):
         err = float(np.abs(f64(a) - b).max())
-        tol = 1e-4 if dtype == torch.float32 else 4e-3 * float(np.abs(b).max()) + 1e-3
+        tol = 1e-4 if dtype == torch.float32 else 1e-2 * float(np.abs(b).max()) + 2e-3
         assert err <= tol, f"{name}: max err {err} > {tol}"
 
 
@@ -45,7 +46,8 @@ def test_backward_fp32(B, H, T, D, W):
     check(B, H, T, D, W, torch.float32, 11 + T + W)
 
 
-@pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 300, 64, 77), (1, 2, 257, 128, 128), (2, 1, 129, 128, 1000)])
+@pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 300, 64, 77), (1, 2, 257, 128, 128), (2, 1, 129, 128, 1000),
+                                       (1, 1, 200, 32, 50), (2, 2, 640, 128, 1), (1, 2, 1000, 64, 300)])
 def test_backward_bf16(B, H, T, D, W):
     check(B, H, T, D, W, torch.bfloat16, 23 + T + W)
 
@@ -84,16 +86,34 @@ def test_backward_deterministic():
     assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
+def test_lse_matches_oracle_weights():
+    """forward_lse's lse is log of the sum of exp(scaled score) over each band."""
+    B, H, T, D, W = 1, 2, 200, 64, 50
+    for dtype in (torch.float32, torch.bfloat16):
+        q, k, v = inputs.prefill_inputs(B, H, T, D, dtype, 47)
+        out, lse = swa.forward_lse(q.to(DEV), k.to(DEV), v.to(DEV), W)
+        swa.device_status()
+        qd, kd = f64(q), f64(k)
+        s = np.einsum("bhid,bhjd->bhij", qd, kd) / np.sqrt(D)
+        i, j = np.arange(T)[:, None], np.arange(T)[None, :]
+        s = np.where((i - j >= 0) & (i - j < W), s, -np.inf)
+        ref = np.log(np.exp(s - s.max(-1, keepdims=True)).sum(-1)) + s.max(-1)
+        tol = 1e-4 if dtype == torch.float32 else 2e-2
+        assert float(np.abs(f64(lse) - ref).max()) <= tol
+        assert torch.equal(out, swa.forward(q.to(DEV), k.to(DEV), v.to(DEV), W))
+
+
 def test_backward_errors():
     lib = _native.lib()
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     t = torch.zeros(1, 1, 16, 513, device=DEV)
     need = lib.swa_backward_workspace_bytes(1, 1, 16)
-    assert need == 16 * 8
+    assert need == 128 * 8  # rows padded to a whole 128-row tile
     ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    lse = torch.zeros(1, 1, 16, device=DEV)
     p, w = t.data_ptr(), ws.data_ptr()
     outs = [torch.empty_like(t).data_ptr() for _ in range(3)]
-    f = lambda *a: lib.swa_backward(p, p, p, p, *outs, *a)
+    f = lambda *a: lib.swa_backward(p, p, p, p, p, lse.data_ptr(), *outs, *a)
     assert f(w, need, 1, 1, 16, 64, 4, 0.125, 0, s) == 0
     assert f(w, need - 8, 1, 1, 16, 64, 4, 0.125, 0, s) == 1     # short workspace
     assert f(w, need, 1, 1, 16, 64, 0, 0.125, 0, s) == 1         # W < 1
