@@ -267,6 +267,8 @@ def main():
     ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--no-module", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-workload", default="mistral",
+                    help="prefill workload whose backward the backward leg times (as --workload)")
     ap.add_argument("--chunk-streams", type=int, default=None,
                     help="override the chunk workload's stream count (smaller profiling runs)")
     ap.add_argument("--workload", default="mistral",
@@ -440,7 +442,7 @@ def main():
     backward_line = None
     if not args.no_backward:
         torch.cuda.empty_cache()
-        bw = inputs.MISTRAL
+        bw = prefill_workload(args.backward_workload)
         bq, bk, bv = (t.to(device) for t in inputs.for_workload(bw))
         gb = torch.Generator().manual_seed(1007)
         bdo = torch.randn(bw.B, bw.H, bw.T, bw.D, generator=gb).to(bw.dtype).to(device)
