@@ -87,10 +87,12 @@ __global__ void __launch_bounds__(256)
 
 // One chunk of 32 columns of one TMEM row: scores s (fp32, raw q.k) and dp, to bf16 P and
 // dS = P (dp - delta): P = exp2(s*c2 - lse2) where the column is valid, else 0. Column
-// t's lse2 and delta come from lse2_of(t), delta_of(t); valid_of(t) masks edge tiles.
-template <bool STORE_P, typename Lse, typename Delta, typename Valid>
+// t's lse2 and delta come from lse2_of(t), delta_of(t). On EDGE tiles only columns
+// cmin..cmax are valid (band membership of one row is an interval of columns); other
+// tiles are valid throughout.
+template <bool STORE_P, bool EDGE, typename Lse, typename Delta>
 __device__ __forceinline__ void bwd_chunk(uint32_t scol, uint32_t dpcol, float c2, Lse lse2_of, Delta delta_of,
-                                          Valid valid_of) {
+                                          int cmin, int cmax) {
     uint32_t s[32], dp[32];
     ptx::tmem_ld32(scol, s);
     ptx::tmem_ld32(dpcol, dp);
@@ -104,7 +106,8 @@ __device__ __forceinline__ void bwd_chunk(uint32_t scol, uint32_t dpcol, float c
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int col = 2 * t + e;
-            const float pe = valid_of(col) ? ptx::ex2(__uint_as_float(s[col]) * c2 - lse2_of(col)) : 0.f;
+            float pe = ptx::ex2(fmaf(__uint_as_float(s[col]), c2, -lse2_of(col)));
+            if (EDGE && !(col >= cmin && col <= cmax)) pe = 0.f;
             p[e] = pe;
             ds[e] = pe * (__uint_as_float(dp[col]) - delta_of(col));
         }
@@ -355,27 +358,32 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             ptx::tc_fence_after();
             const bool edge = k != 2;
-#pragma unroll 1
+            // valid columns of this row in the tile, as an interval of tile columns
+            int clo, chi;
+            if (KV) {  // row = key xr, columns = queries: xr <= i <= min(xr + W - 1, T - 1)
+                clo = xr - 128 * yt;
+                chi = (xr < T ? min(xr + W - 1, T - 1) : -1) - 128 * yt;
+            } else {   // row = query xr, columns = keys: max(0, xr - W + 1) <= j <= min(xr, T - 1)
+                clo = max(0, xr - W + 1) - 128 * yt;
+                chi = (xr < T ? xr : -1) - 128 * yt;
+                if (xr >= T) clo = chi + 1;
+            }
+            if (KV && xr >= T) clo = chi + 1;
+#pragma unroll 2
             for (int cc = 0; cc < 4; ++cc) {
-                const int y0 = 128 * yt + 32 * cc;  // index of this chunk's first column
+                const uint32_t sc = tl + Cf::kColS + 32 * cc, dc = tl + Cf::kColDP + 32 * cc;
+                const int cmin = clo - 32 * cc, cmax = chi - 32 * cc;
                 if (KV) {
-                    // row = key j = xr, columns = queries i = y0 + t: valid iff 0 <= i - j < W, i < T
-                    auto lse_of = [&](int t) { return sts[32 * cc + t]; };
-                    auto delta_of = [&](int t) { return sts[128 + 32 * cc + t]; };
-                    auto valid = [&](int t) {
-                        const int d = y0 + t - xr;
-                        return !edge || (d >= 0 && d < W && y0 + t < T && xr < T);
-                    };
-                    bwd_chunk<true>(tl + Cf::kColS + 32 * cc, tl + Cf::kColDP + 32 * cc, c2, lse_of, delta_of, valid);
+                    const float* sl = sts + 32 * cc;
+                    auto lse_of = [&](int t) { return sl[t]; };
+                    auto delta_of = [&](int t) { return sl[128 + t]; };
+                    if (edge) bwd_chunk<true, true>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
+                    else bwd_chunk<true, false>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
                 } else {
-                    // row = query i = xr, columns = keys j = y0 + t
                     auto lse_of = [&](int) { return my_lse2; };
                     auto delta_of = [&](int) { return my_delta; };
-                    auto valid = [&](int t) {
-                        const int d = xr - (y0 + t);
-                        return !edge || (d >= 0 && d < W && y0 + t < T && xr < T);
-                    };
-                    bwd_chunk<false>(tl + Cf::kColS + 32 * cc, tl + Cf::kColDP + 32 * cc, c2, lse_of, delta_of, valid);
+                    if (edge) bwd_chunk<false, true>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
+                    else bwd_chunk<false, false>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
                 }
             }
             ptx::tmem_st_wait();
