@@ -11,8 +11,8 @@
 //                     (padding rows get lse = +inf, delta = 0, so they weigh nothing).
 //   bwd_kv_kernel<D>  one CTA per (b, h, 128-key tile): K and V stay in shared memory;
 //                     for every query tile that meets the band, TMA brings Q, dO and the
-//                     tile's (lse, delta); S^T = K Q^T and dP^T = V dO^T go to TMEM; four
-//                     warps (one key row each) turn them into bf16 P^T and dS^T over the
+//                     tile's (lse, delta); S^T = K Q^T and dP^T = V dO^T go to TMEM; eight
+//                     warps (two per key row, 64 columns each) turn them into bf16 P^T and dS^T over the
 //                     same TMEM columns; then dV += P^T dO and dK += dS^T Q accumulate in
 //                     TMEM (TS form: A from TMEM, B from shared memory).
 //   bwd_q_kernel<D>   one CTA per (b, h, 128-query tile): Q and dO stay; for every key
@@ -33,7 +33,8 @@
 
 namespace swa {
 
-constexpr int kBwdTcThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 element-wise
+constexpr int kBwdTcThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2..9 element-wise
+constexpr int kBwdTcEw = 256;       // element-wise threads: two warps per row quarter
 
 template <int D>
 struct BwdTcCfg {
@@ -196,10 +197,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(stat_full + x, 1);
-            ptx::mbar_init(stat_empty + x, 128);
+            ptx::mbar_init(stat_empty + x, kBwdTcEw);
         }
         ptx::mbar_init(s_full, 1);
-        ptx::mbar_init(p_full, 128);
+        ptx::mbar_init(p_full, kBwdTcEw);
         ptx::mbar_init(o_final, 1);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -338,7 +339,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
     } else {
         // -------------------------------------------------------------------- element-wise
+        // warps 2..9: warp w serves TMEM lanes 32*(w%4).. and column chunks 2*half, 2*half+1
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;  // the TMEM lane = this thread's resident row
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
         const int xr = 128 * xt + r;         // key index (KV) or query index (Q)
@@ -369,8 +372,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 if (xr >= T) clo = chi + 1;
             }
             if (KV && xr >= T) clo = chi + 1;
-#pragma unroll 2
-            for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+            for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
                 const uint32_t sc = tl + Cf::kColS + 32 * cc, dc = tl + Cf::kColDP + 32 * cc;
                 const int cmin = clo - 32 * cc, cmax = chi - 32 * cc;
                 if (KV) {
@@ -400,11 +403,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             ptx::tc_fence_after();
             const bool live = xr < T;
             const int64_t row = ((int64_t)bh * T + xr) * D;
+            // each of the two warps of a quarter stores half of the D columns
+            const int dh = (D / 2) * half;
             if (KV) {
-                bwd_store_row<D>(tl + Cf::kColB, c, g1 + row, live);    // dK = c dS^T Q
-                bwd_store_row<D>(tl + Cf::kColA, 1.f, g2 + row, live);  // dV = P^T dO
+                bwd_store_row<D / 2>(tl + Cf::kColB + dh, c, g1 + row + dh, live);    // dK = c dS^T Q
+                bwd_store_row<D / 2>(tl + Cf::kColA + dh, 1.f, g2 + row + dh, live);  // dV = P^T dO
             } else {
-                bwd_store_row<D>(tl + Cf::kColA, c, g1 + row, live);    // dQ = c dS K
+                bwd_store_row<D / 2>(tl + Cf::kColA + dh, c, g1 + row + dh, live);    // dQ = c dS K
             }
         } else {
             atomicCAS(status, 0, 5);
