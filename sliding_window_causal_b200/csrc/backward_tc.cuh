@@ -12,9 +12,11 @@
 //   bwd_kv_kernel<D>  one CTA per (b, h, 128-key tile): K and V stay in shared memory;
 //                     for every query tile that meets the band, TMA brings Q, dO and the
 //                     tile's (lse, delta); S^T = K Q^T and dP^T = V dO^T go to TMEM; eight
-//                     warps (two per key row, 64 columns each) turn them into bf16 P^T and dS^T over the
-//                     same TMEM columns; then dV += P^T dO and dK += dS^T Q accumulate in
-//                     TMEM (TS form: A from TMEM, B from shared memory).
+//                     warps (two per key row, 64 columns each) turn them into bf16 P^T and
+//                     dS^T over the dP^T columns; then dV += P^T dO and dK += dS^T Q
+//                     accumulate in TMEM (TS form: A from TMEM, B from shared memory). The
+//                     next tile's S^T is computed while the element-wise warps work: they
+//                     read their scores into registers first and release the S columns.
 //   bwd_q_kernel<D>   one CTA per (b, h, 128-query tile): Q and dO stay; for every key
 //                     tile of the band S = Q K^T and dP = dO V^T, then dS (bf16, in TMEM)
 //                     and dQ += dS K.
@@ -49,8 +51,8 @@ struct BwdTcCfg {
     static constexpr int kStatOff = kRingOff + kStages * kTileBytes;
     static constexpr int kBarOff = kStatOff + kStatStages * kStatBytes;
     // fix_full, ring_full[S], ring_empty[S], stat_full[2], stat_empty[2], s_full, p_full,
-    // o_final, drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4;
+    // o_final, drain, s_read
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 5;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static constexpr uint32_t kTmemCols = 512;
@@ -86,20 +88,16 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// One chunk of 32 columns of one TMEM row: scores s (fp32, raw q.k) and dp, to bf16 P and
-// dS = P (dp - delta): P = exp2(s*c2 - lse2) where the column is valid, else 0. Column
-// t's lse2 and delta come from lse2_of(t), delta_of(t). On EDGE tiles only columns
-// cmin..cmax are valid (band membership of one row is an interval of columns); other
-// tiles are valid throughout.
+// One chunk of 32 columns of one TMEM row, already in registers: scores s (fp32, raw q.k)
+// and dp, to bf16 P and dS = P (dp - delta), with P = exp2(s*c2 - lse2) where the column
+// is valid, else 0. Column t's lse2 and delta come from lse2_of(t), delta_of(t). On EDGE
+// tiles only columns cmin..cmax are valid (band membership of one row is an interval of
+// columns); other tiles are valid throughout. dS goes to columns dpcol .. dpcol+15 and,
+// when STORE_P, P to dpcol+16 .. dpcol+31 (both over dp values already read), leaving the
+// S columns free for the next tile's scores.
 template <bool STORE_P, bool EDGE, typename Lse, typename Delta>
-__device__ __forceinline__ void bwd_chunk(uint32_t scol, uint32_t dpcol, float c2, Lse lse2_of, Delta delta_of,
-                                          int cmin, int cmax) {
-    uint32_t s[32], dp[32];
-    ptx::tmem_ld32(scol, s);
-    ptx::tmem_ld32(dpcol, dp);
-    ptx::tmem_ld_wait();
-    ptx::reg_fence(s);
-    ptx::reg_fence(dp);
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], uint32_t dpcol,
+                                          float c2, Lse lse2_of, Delta delta_of, int cmin, int cmax) {
     uint32_t ph[16], dh[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
@@ -115,8 +113,8 @@ __device__ __forceinline__ void bwd_chunk(uint32_t scol, uint32_t dpcol, float c
         ph[t] = ptx::pack_bf16x2(p[0], p[1]);
         dh[t] = ptx::pack_bf16x2(ds[0], ds[1]);
     }
-    if (STORE_P) ptx::tmem_st16(scol, ph);
-    ptx::tmem_st16(STORE_P ? dpcol : scol, dh);
+    ptx::tmem_st16(dpcol, dh);
+    if (STORE_P) ptx::tmem_st16(dpcol + 16, ph);
 }
 
 // Store one 128-column TMEM accumulator row (D fp32 values from column col) times a, as
@@ -168,6 +166,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     uint64_t* p_full = s_full + 1;
     uint64_t* o_final = p_full + 1;
     uint64_t* drain = o_final + 1;
+    uint64_t* s_read = drain + 1;  // the element-wise warps have read S and dP of a tile
     const float* st_smem = reinterpret_cast<const float*>(smem + Cf::kStatOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cf::kMiscOff + 4);
@@ -203,6 +202,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         ptx::mbar_init(p_full, kBwdTcEw);
         ptx::mbar_init(o_final, 1);
         ptx::mbar_init(drain, 1);
+        ptx::mbar_init(s_read, kBwdTcEw);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -282,54 +282,90 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const uint32_t ring_lo = ptx::smem_u32(smem + Cf::kRingOff) >> 4;
             constexpr uint32_t kStageLo = Cf::kTileBytes >> 4;
             bool ok = ptx::mbar_wait(fix_full, 0, wait_limit_ns, abort_flag);
-            uint32_t L = 0;
-            int j = 0;  // visited tiles
-            for (int yt = lo; yt <= hi && ok; ++yt) {
-                if (cls(yt) == 0) continue;
-                const uint32_t sta = L % NS, stb = (L + 1) % NS;
-                ok = ptx::mbar_wait(ring_full + sta, (L / NS) & 1, wait_limit_ns, abort_flag);
-                if (ok) ok = ptx::mbar_wait(ring_full + stb, ((L + 1) / NS) & 1, wait_limit_ns, abort_flag);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint32_t a_lo = ring_lo + sta * kStageLo, b_lo = ring_lo + stb * kStageLo;
-                // KV: S^T = K Q^T, dP^T = V dO^T.   Q: S = Q K^T, dP = dO V^T.
+            auto next_visited = [&](int y) {  // the first visited tile after y (> hi if none)
+                for (++y; y <= hi && cls(y) == 0; ++y) {
+                }
+                return y;
+            };
+            auto wait_stage = [&](uint32_t idx) {
+                return ptx::mbar_wait(ring_full + idx % NS, (idx / NS) & 1, wait_limit_ns, abort_flag);
+            };
+            // KV: S^T = K Q^T, dP^T = V dO^T.   Q: S = Q K^T, dP = dO V^T.
+            // Tile j's streamed operands sit in stages L % NS (a: Q or K) and (L+1) % NS (b: dO or V).
+            auto issue_s = [&](uint32_t Lj) {
+                const uint32_t a_lo = ring_lo + (Lj % NS) * kStageLo;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
                     ptx::mma_ss(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k), desc_hi | ((a_lo + off) | lo_k),
                                 idesc_s, kk > 0 ? 1u : 0u);
                 }
+            };
+            auto issue_dp = [&](uint32_t Lj) {
+                const uint32_t b_lo = ring_lo + ((Lj + 1) % NS) * kStageLo;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
                     ptx::mma_ss(tmem + Cf::kColDP, desc_hi | ((fb_lo + off) | lo_k), desc_hi | ((b_lo + off) | lo_k),
                                 idesc_s, kk > 0 ? 1u : 0u);
                 }
+            };
+            uint32_t L = 0;
+            int j = 0;  // visited tiles
+            int yt = next_visited(lo - 1);
+            if (ok) ok = wait_stage(0) && wait_stage(1);
+            if (ok) {
+                ptx::tc_fence_after();
+                issue_s(0);
+                issue_dp(0);
                 ptx::tc_commit(s_full);
-                ok = ptx::mbar_wait(p_full, j & 1, wait_limit_ns, abort_flag);
+            }
+            while (ok) {
+                const int ynext = next_visited(yt);
+                // the next tile's scores as soon as this tile's S and dP are in registers
+                ok = ptx::mbar_wait(s_read, j & 1, wait_limit_ns, abort_flag);
+                if (ok && ynext <= hi) {
+                    ok = wait_stage(L + 2);
+                    if (ok) {
+                        ptx::tc_fence_after();
+                        issue_s(L + 2);
+                    }
+                }
+                if (ok) ok = ptx::mbar_wait(p_full, j & 1, wait_limit_ns, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                const uint32_t sta = L % NS, stb = (L + 1) % NS;
+                const uint32_t a_lo = ring_lo + sta * kStageLo, b_lo = ring_lo + stb * kStageLo;
                 if (KV) {
-                    // dV += P^T dO (B = dO, the streamed b tile); dK += dS^T Q (B = Q, the streamed a tile)
+                    // dV += P^T dO (A = P^T, the +16 half of each dP chunk; B = dO);
+                    // dK += dS^T Q (A = dS^T, the first half; B = Q)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColS + pp_pcol(kk),
+                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk) + 16,
                                     desc_hi | ((b_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         ptx::mma_ts(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
                                     desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 } else {
-                    // dQ += dS K (A = dS over the S columns, B = K, the streamed a tile)
+                    // dQ += dS K (A = dS in the dP columns, B = K)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColS + pp_pcol(kk),
+                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk),
                                     desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 ptx::tc_commit(ring_empty + sta);
                 ptx::tc_commit(ring_empty + stb);
+                if (ynext > hi) break;
+                // the next tile's dP, over this tile's P and dS, after the products above read them
+                ok = wait_stage(L + 3);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_dp(L + 2);
+                ptx::tc_commit(s_full);
                 L += 2;
                 ++j;
+                yt = ynext;
             }
             if (ok) ptx::tc_commit(o_final);
             if (!ok) {
@@ -372,21 +408,35 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 if (xr >= T) clo = chi + 1;
             }
             if (KV && xr >= T) clo = chi + 1;
+            // the scores first, so that the S columns can take the next tile's scores
+            uint32_t sv[2][32];
 #pragma unroll
-            for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-                const uint32_t sc = tl + Cf::kColS + 32 * cc, dc = tl + Cf::kColDP + 32 * cc;
+            for (int x = 0; x < 2; ++x) ptx::tmem_ld32(tl + Cf::kColS + 32 * (2 * half + x), sv[x]);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 2; ++x) ptx::reg_fence(sv[x]);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(s_read);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int cc = 2 * half + x;
+                const uint32_t dc = tl + Cf::kColDP + 32 * cc;
+                uint32_t dpv[32];
+                ptx::tmem_ld32(dc, dpv);
+                ptx::tmem_ld_wait();
+                ptx::reg_fence(dpv);
                 const int cmin = clo - 32 * cc, cmax = chi - 32 * cc;
                 if (KV) {
                     const float* sl = sts + 32 * cc;
                     auto lse_of = [&](int t) { return sl[t]; };
                     auto delta_of = [&](int t) { return sl[128 + t]; };
-                    if (edge) bwd_chunk<true, true>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
-                    else bwd_chunk<true, false>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
+                    if (edge) bwd_chunk<true, true>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
+                    else bwd_chunk<true, false>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
                 } else {
                     auto lse_of = [&](int) { return my_lse2; };
                     auto delta_of = [&](int) { return my_delta; };
-                    if (edge) bwd_chunk<false, true>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
-                    else bwd_chunk<false, false>(sc, dc, c2, lse_of, delta_of, cmin, cmax);
+                    if (edge) bwd_chunk<false, true>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
+                    else bwd_chunk<false, false>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
                 }
             }
             ptx::tmem_st_wait();
