@@ -166,6 +166,23 @@ def dist_setup(args):
     return world, rank, local, pg
 
 
+def max_over_ranks(x, pg, device):
+    """The largest of every rank's x (x itself without a process group); all ranks must
+    call it, in the same order."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    pg.barrier()
+    return t.item()
+
+
+def whole_job(units_per_rank, ms_per_step, world):
+    """Whole-job throughput under weak scaling: every rank processes units_per_rank per
+    step, and the step takes ms_per_step (the max over ranks)."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def timed(fn, steps, stream, pg, device):
     """Run fn() `steps` times between a barrier + synchronize on both sides; returns
     the elapsed device time in ms (CUDA events on `stream`), max over ranks."""
@@ -178,13 +195,7 @@ def timed(fn, steps, stream, pg, device):
         fn()
     end.record(stream)
     torch.cuda.synchronize(device)
-    ms = start.elapsed_time(end)
-    if pg is not None:
-        t = torch.tensor([ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        pg.barrier()
-        ms = t.item()
-    return ms
+    return max_over_ranks(start.elapsed_time(end), pg, device)
 
 
 def cpu_baseline_prefill(wl, budget_s, q, k, v):
@@ -310,7 +321,7 @@ def main():
         ms = timed(fwd, args.steps, stream, pg, device)
     swa.device_status()
     ms_step = ms / args.steps
-    value = world * F / (ms_step * 1e-3) / 1e12
+    value = whole_job(F, ms_step, world) / 1e12
     achieved = F / (ms_step * 1e-3) / 1e12
 
     # ------------------------------------------------------------ e2e (host buffers)
