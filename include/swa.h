@@ -30,7 +30,8 @@
  *    status word and reported by swa_device_status().
  *  - `out` must not alias q, k, v (or the rings); this is documented, not checked.
  *  - Results are deterministic: the same inputs and sizes give bitwise-identical
- *    outputs on every run.
+ *    outputs on every run (swa_mha_forward: its attention is; its projections are as
+ *    reproducible as the GEMM algorithm cuBLASLt picks).
  */
 #ifndef SWA_H
 #define SWA_H
