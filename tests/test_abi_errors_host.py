@@ -1,0 +1,97 @@
+"""Argument validation at the C ABI, on the CPU: every call checks its arguments before it
+touches the device, so a refused call returns its status here without a GPU. The pointers
+are dummies that a valid call would have to dereference; every call here is refused or is
+a no-op (an empty batch), so none of them launches anything, on a machine with a GPU too."""
+import ctypes
+
+import pytest
+
+from sliding_window_causal_b200 import _native, build
+
+DUMMY = 0x10000  # 64 KiB-aligned, never dereferenced
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.lib()
+
+
+def strides(*vals):
+    return (ctypes.c_int64 * len(vals))(*vals)
+
+
+def test_forward_errors(lib):
+    p = DUMMY
+    f = lib.swa_forward
+    assert f(p, p, p, p, 1, 2, 8, 64, 0, 1, None) == INVALID       # W < 1
+    assert f(p, p, p, p, 1, -2, 8, 64, 4, 1, None) == INVALID      # negative size
+    assert f(p, p, p, p, 1, 2, 8, 0, 4, 1, None) == INVALID        # D < 1
+    assert f(p, p, p, p, 1, 2, 8, 64, 4, 7, None) == INVALID       # dtype
+    assert f(None, p, p, p, 1, 2, 8, 64, 4, 1, None) == INVALID    # null pointer
+    assert f(p, p, p, p, 1, 2, 8, 64, 4, 7, None) == INVALID
+    assert lib.swa_last_error()                                     # a refusal leaves a message
+    assert f(None, None, None, None, 0, 2, 8, 64, 4, 1, None) == OK  # empty: no-op
+
+
+def test_forward_ex_errors(lib):
+    p = DUMMY
+    f = lib.swa_forward_ex
+    good = strides(*([2 * 8 * 64, 8 * 64, 64] * 4))
+    assert f(p, p, p, p, 1, 2, 8, 64, 4, float("nan"), good, 1, None) == INVALID
+    assert f(p, p, p, p, 1, 2, 8, 64, 4, float("inf"), good, 1, None) == INVALID
+    neg = strides(*([2 * 8 * 64, -8 * 64, 64] + [2 * 8 * 64, 8 * 64, 64] * 3))
+    assert f(p, p, p, p, 1, 2, 8, 64, 4, 0.125, neg, 1, None) == INVALID
+    huge = strides(*([1 << 39, 8 * 64, 64] + [2 * 8 * 64, 8 * 64, 64] * 3))
+    assert f(p, p, p, p, 2, 2, 8, 64, 4, 0.125, huge, 1, None) == INVALID
+    assert b"stride" in lib.swa_last_error()
+
+
+def test_band_weights_errors(lib):
+    p = DUMMY
+    f = lib.swa_band_weights
+    assert f(p, p, p, 1, 2, 8, 64, 0, 0.1, None, 1, None) == INVALID
+    assert f(p, p, None, 1, 2, 8, 64, 4, 0.1, None, 1, None) == INVALID
+    assert f(p, p, p, 1, 2, 8, 64, 4, float("nan"), None, 1, None) == INVALID
+    assert f(p, p, p, 1, 2, 8, 5000, 4, 0.1, None, 0, None) == UNSUPPORTED  # D > 4096
+
+
+def test_decode_and_streaming_errors(lib):
+    p = DUMMY
+    for f in (lib.swa_decode, lib.swa_decode_noalloc):
+        assert f(p, p, p, p, p, 2, 2, 64, 0, None) == INVALID           # W < 1
+        assert f(p, p, p, p, p, 2, 2, 96, 16, None) == UNSUPPORTED      # D = 96
+        assert f(p + 2, p, p, p, p, 2, 2, 64, 16, None) == MISALIGNED   # q not 16-byte aligned
+        assert f(p, p, p, None, p, 2, 2, 64, 16, None) == INVALID       # null pos
+        assert f(p, p, p, p, p, 0, 2, 64, 16, None) == OK               # no streams: no-op
+    c = lib.swa_chunk_forward
+    assert c(p, p, p, p, p, p, p, 1, 1, 8, 64, 0, None) == INVALID
+    assert c(p, p, p, p, p, p, p, 1, 1, 8, 96, 16, None) == UNSUPPORTED
+    assert c(p, p, p, p + 8, p, p, p, 1, 1, 8, 64, 16, None) == MISALIGNED
+    assert c(p, p, p, p, p, p, p, 1, 1, 0, 64, 16, None) == OK         # empty chunk
+    a = lib.swa_ring_append
+    assert a(p, p, p, p, p, 1, 1, 8, 64, 0, None) == INVALID
+    assert a(p, p, p, p, None, 1, 1, 8, 64, 16, None) == INVALID
+
+
+def test_module_and_backward_errors(lib):
+    p = DUMMY
+    need = lib.swa_mha_workspace_bytes(1, 8, 128, 1)
+    m = lambda *a: lib.swa_mha_forward(p, p, None, p, None, p, None, p, None, p, *a)
+    assert m(p, need, 1, 8, 128, 3, 4, 1, None) == INVALID        # d_model % H
+    assert m(p, need, 1, 8, 128, 4, 4, 1, None) == UNSUPPORTED    # bf16 head width 32
+    assert m(p, need - 1, 1, 8, 128, 1, 4, 1, None) == INVALID    # short workspace
+    assert m(p + 16, need, 1, 8, 128, 1, 4, 1, None) == MISALIGNED
+    assert m(p, need, 1, 8, 128, 1, 4, 9, None) == INVALID        # dtype
+    wb = lib.swa_backward_workspace_bytes(1, 1, 16)
+    b = lambda *a: lib.swa_backward(p, p, p, p, p, p, p, p, p, *a)
+    assert b(p, wb - 8, 1, 1, 16, 64, 4, 0.125, 1, None) == INVALID   # short workspace
+    assert b(p, wb, 1, 1, 16, 64, 0, 0.125, 1, None) == INVALID       # W < 1
+    assert b(p, wb, 1, 1, 16, 64, 4, float("nan"), 1, None) == INVALID
+    assert b(p, wb, 1, 1, 16, 513, 4, 0.125, 0, None) == UNSUPPORTED  # CUDA-core D limit
+    assert b(p + 64, wb, 1, 1, 16, 64, 4, 0.125, 1, None) == MISALIGNED  # bf16 workspace 256
+    assert b(p, wb, 1, 1, 16, 64, 4, -0.5, 1, None) == UNSUPPORTED    # bf16 scale > 0
+    lse_none = lib.swa_backward(p, p, p, p, p, None, p, p, p, p, wb, 1, 1, 16, 64, 4, 0.125, 1, None)
+    assert lse_none == INVALID                                        # tensor-core path needs lse
+    assert lib.swa_forward_lse(p, p, p, p, None, 1, 1, 16, 64, 4, 0.125, 1, None) == INVALID
