@@ -233,7 +233,8 @@ int64_t swa_mha_workspace_bytes(int64_t B, int64_t T, int64_t d_model, int dtype
  * swa_forward_lse: swa_forward (contiguous operands, the given scale) that also writes the
  * natural log-sum-exp of every row's scaled scores, the statistic swa_backward needs:
  *   lse[b,h,i] = log( sum_{j in band(i)} exp(scale * q_i . k_j) )    [B, H, T] fp32.
- * Errors: as swa_forward_ex; a null lse -> SWA_ERR_INVALID_ARG.
+ * Errors: as swa_forward_ex; a null lse (for a non-empty batch) -> SWA_ERR_INVALID_ARG,
+ * an lse not 4-byte aligned -> SWA_ERR_MISALIGNED.
  */
 int swa_forward_lse(const void* q, const void* k, const void* v, void* out, float* lse,
                     int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, double scale,
@@ -260,8 +261,14 @@ int swa_forward_lse(const void* q, const void* k, const void* v, void* out, floa
  *                   scale must be > 0. Other cases (SWA_F32, or bf16 with another D) run
  *                   in fp32 on the CUDA cores, D <= 512, recomputing the statistics
  *                   (out and lse are then not read and may be NULL).
- * There are no atomics: the results are deterministic. Errors: as swa_forward_ex, plus a
- * short workspace -> SWA_ERR_INVALID_ARG.
+ * There are no atomics: the results are deterministic. Errors (nothing is enqueued):
+ *   invalid sizes, dtype or scale, a null pointer (out and lse included on the tensor-core
+ *   path) or a workspace shorter than swa_backward_workspace_bytes -> SWA_ERR_INVALID_ARG;
+ *   tensor-core path: tensors not 16-byte aligned, workspace not 256-byte aligned or lse
+ *   not 4-byte aligned -> SWA_ERR_MISALIGNED, scale <= 0 -> SWA_ERR_UNSUPPORTED;
+ *   CUDA-core path: D > 512 -> SWA_ERR_UNSUPPORTED, tensors not aligned to their element
+ *   size or workspace not 8-byte aligned -> SWA_ERR_MISALIGNED.
+ * B, H or T = 0 is a no-op that returns SWA_OK.
  */
 int swa_backward(const void* q, const void* k, const void* v, const void* out,
                  const void* dout, const float* lse, void* dq, void* dk, void* dv,

@@ -95,3 +95,6 @@ def test_module_and_backward_errors(lib):
     lse_none = lib.swa_backward(p, p, p, p, p, None, p, p, p, p, wb, 1, 1, 16, 64, 4, 0.125, 1, None)
     assert lse_none == INVALID                                        # tensor-core path needs lse
     assert lib.swa_forward_lse(p, p, p, p, None, 1, 1, 16, 64, 4, 0.125, 1, None) == INVALID
+    assert lib.swa_forward_lse(p, p, p, p, p + 2, 1, 1, 16, 64, 4, 0.125, 1, None) == MISALIGNED
+    assert b(p + 2, wb, 1, 1, 16, 64, 4, 0.125, 0, None) == MISALIGNED  # fp32 workspace 8
+    assert b(p, wb, 0, 1, 16, 64, 4, 0.125, 1, None) == OK              # empty batch: no-op
