@@ -8,10 +8,10 @@
  *   band(i)      = { j : max(0, i-W+1) <= j <= i }
  *
  * Sources: "27. Sliding-Window Attention" (Problem; Step-by-Step Approach steps 1-5:
- * scaled scores, the band mask (j <= i) & (i - j < window_size), -inf masking,
- * softmax over keys, weights @ v); "25. Sliding-Window Causal Attention for
- * Streaming Inference" (Step-by-Step Approach step 3, the strict lower bound
- * key_pos > query_pos - window_size); "NNX Sliding-Window Attention" (opening
+ * scaled scores, a mask that keeps j <= i with i - j below the window, -inf outside it,
+ * a softmax over the keys, then the weighted sum of v); "25. Sliding-Window Causal
+ * Attention for Streaming Inference" (Step-by-Step Approach step 3: the oldest key kept
+ * is strictly newer than i - W); "NNX Sliding-Window Attention" (opening
  * paragraph: keys max(0, i-W+1) .. i; W = 1 is self-attention only; W >= T is
  * ordinary causal attention). The one-key-wider interval [i-W, i] of "Sliding
  * Window Attention" (Mathematical Formulation and Attention Masking) is not
@@ -77,9 +77,9 @@ int swa_forward(const void* q, const void* k, const void* v, void* out,
 /*
  * swa_forward_ex: swa_forward with a caller-chosen score scale and strided operands.
  *
- * "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2) takes its
- * inputs as (batch, seq_len, num_heads, head_dim) and an optional scale that defaults to
- * 1/sqrt(head_dim). This call covers both:
+ * "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2) lays its
+ * inputs out batch, position, head, feature ([B,T,H,D]) and lets the caller choose the
+ * score scale, 1/sqrt(D) when none is given. This call covers both:
  *   scale   : scores are (q . k) * scale. swa_forward is scale = 1/sqrt(D). SWA_BF16 takes
  *             any scale > 0 (the tensor-core softmax scales the row maximum of the raw
  *             scores, which is the maximum of the scaled ones only for a positive scale);

@@ -9,11 +9,11 @@
  * or reordering. For every batch b, head h and query position i:
  *
  *   band(i) = { j : max(0, i-W+1) <= j <= i }
- *       "27. Sliding-Window Attention", Step-by-Step Approach, step 2: the band
- *       mask is (j <= i) & (i - j < window_size).
+ *       "27. Sliding-Window Attention", Step-by-Step Approach, step 2: a key is
+ *       kept when it is not after the query and fewer than W positions behind it.
  *       "25. Sliding-Window Causal Attention for Streaming Inference",
- *       Step-by-Step Approach, step 3: key_pos <= query_pos and
- *       key_pos > query_pos - window_size.
+ *       Step-by-Step Approach, step 3: the same two bounds, the lower one strict
+ *       (j > i - W).
  *       "NNX Sliding-Window Attention", opening paragraph: keys from
  *       max(0, i - W + 1) through i.
  *   s_j    = (sum_d q[b,h,i,d] * k[b,h,j,d]) / sqrt(D)       for j in band(i)
@@ -33,7 +33,8 @@
  *
  * Layout: every tensor is row-major contiguous [B, H, T, D], so element
  * (b,h,t,d) sits at ((b*H + h)*T + t)*D + d ("27. Sliding-Window Attention",
- * reference solution: q has shape (batch, heads, seq, head_dim)).
+ * reference solution: the queries are laid out batch, then head, then position, then
+ * feature).
  *
  * Decode: the rolling buffer keeps the last W positions of each stream. Position
  * p lives in slot p mod W ("25. Sliding-Window Causal Attention for Streaming
@@ -43,7 +44,7 @@
  *
  * Scale: the *_scaled entry points multiply the dot products by a caller-given
  * factor instead of 1/sqrt(D) ("Mistral Architecture > Implementation: Sliding
- * Window Attention", Step 2: an optional scale that defaults to 1/sqrt(head_dim)).
+ * Window Attention", Step 2: the caller may pass the scale; 1/sqrt(D) when absent).
  * The plain entry points are those with scale = 1/sqrt(D).
  *
  * Return codes: 0 on success, 1 for an invalid argument (W < 1, a negative size,
