@@ -217,7 +217,10 @@ int swa_ring_append(const void* k, const void* v, void* kring, void* vring, cons
  * q, k, v in place as [B, T, H, Dh] (no transposes). All work is enqueued on `stream`.
  * Errors: as swa_forward_ex, plus d_model % H != 0 or a short workspace ->
  * SWA_ERR_INVALID_ARG, pointers not 16-byte aligned (workspace 256) -> SWA_ERR_MISALIGNED,
- * a GEMM library failure -> SWA_ERR_CUDA. B*T == 0 -> SWA_OK with nothing enqueued.
+ * a GEMM library failure -> SWA_ERR_CUDA. B*T == 0 -> SWA_OK with nothing enqueued. Every
+ * refusal, the attention's included, is decided before the first GEMM is enqueued; only
+ * a CUDA or GEMM-library failure can come after earlier steps were enqueued, and out is
+ * then undefined.
  */
 int swa_mha_forward(const void* x, const void* wq, const void* bq, const void* wk, const void* bk,
                     const void* wv, const void* bv, const void* wo, const void* bo, void* out,

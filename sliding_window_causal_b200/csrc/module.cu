@@ -169,26 +169,30 @@ int swa_mha_forward(const void* x, const void* wq, const void* bq, const void* w
     if (dtype == SWA_BF16 && d_model % 8 != 0)
         return fail(SWA_ERR_MISALIGNED, "%s: bf16 d_model must be a multiple of 8", fn);
 
+    const int64_t M = B * T;
+    const size_t part = round256((size_t)(M * d_model) * esz);
+    char* base = static_cast<char*>(workspace);
+    void *q = base, *k = base + part, *v = base + 2 * part, *attn = base + 3 * part, *lt_ws = base + 4 * part;
+    // [B*T, d] is [B, T, H, Dh]: element strides b = T*d, h = Dh, t = d for every operand
+    const int64_t st[12] = {T * d_model, Dh, d_model, T * d_model, Dh, d_model,
+                            T * d_model, Dh, d_model, T * d_model, Dh, d_model};
+    const double scale = 1.0 / std::sqrt((double)Dh);
+    // the attention's own refusals come before the first GEMM is enqueued
+    int64_t eff[4][3];
+    if (int rc = swa_internal::check_forward(fn, q, k, v, attn, B, H, T, Dh, W, scale, st, dtype, eff)) return rc;
+
     int dev;
     cudaError_t ce = cudaGetDevice(&dev);
     if (ce != cudaSuccess) return fail(SWA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(ce));
     cublasLtHandle_t h;
     if (int rc = lt_handle(dev, &h)) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int64_t M = B * T;
-    const size_t part = round256((size_t)(M * d_model) * esz);
-    char* base = static_cast<char*>(workspace);
-    void *q = base, *k = base + part, *v = base + 2 * part, *attn = base + 3 * part, *lt_ws = base + 4 * part;
     int rc;
     if ((rc = gemm(dev, h, dtype, x, wq, bq, q, M, d_model, d_model, lt_ws, s)) ||
         (rc = gemm(dev, h, dtype, x, wk, bk, k, M, d_model, d_model, lt_ws, s)) ||
         (rc = gemm(dev, h, dtype, x, wv, bv, v, M, d_model, d_model, lt_ws, s)))
         return rc;
-    // [B*T, d] is [B, T, H, Dh]: element strides b = T*d, h = Dh, t = d for every operand
-    const int64_t st[12] = {T * d_model, Dh, d_model, T * d_model, Dh, d_model,
-                            T * d_model, Dh, d_model, T * d_model, Dh, d_model};
-    if ((rc = swa_forward_ex(q, k, v, attn, B, H, T, Dh, W, 1.0 / std::sqrt((double)Dh), st, dtype, stream)))
-        return rc;
+    if ((rc = swa_forward_ex(q, k, v, attn, B, H, T, Dh, W, scale, st, dtype, stream))) return rc;
     if ((rc = gemm(dev, h, dtype, attn, wo, bo, out, M, d_model, d_model, lt_ws, s))) return rc;
     return swa_internal::clear_error();
 }

@@ -312,19 +312,17 @@ int check_sizes(const char* fn, int64_t B, int64_t H, int64_t T, int64_t D, int6
     return SWA_OK;
 }
 
-int forward_impl(const char* fn, const void* q, const void* k, const void* v, void* out, int64_t B,
-                 int64_t H, int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides,
-                 int dtype, void* stream, float* lse = nullptr) {
-    if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
-    if (B == 0 || H == 0 || T == 0) return success();
-    if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
-    int64_t st[4][3];
-    if (int rc = read_strides(fn, strides, 4, B, H, T, D, st)) return rc;
-    const int Wi = (int)(W < T ? W : T);  // W >= T is causal attention
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    DeviceState* ds;
-    if (int rc = device_state(&ds)) return rc;
+}  // namespace
 
+namespace swa_internal {
+
+int check_forward(const char* fn, const void* q, const void* k, const void* v, const void* out, int64_t B,
+                  int64_t H, int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides, int dtype,
+                  int64_t st[4][3]) {
+    if (int rc = check_sizes(fn, B, H, T, D, W, dtype, scale)) return rc;
+    if (B == 0 || H == 0 || T == 0) return SWA_OK;
+    if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (int rc = read_strides(fn, strides, 4, B, H, T, D, st)) return rc;
     if (dtype == SWA_BF16) {
         if (D != 64 && D != 128)
             return fail(SWA_ERR_UNSUPPORTED, "%s: bf16 needs D = 64 or 128 (got %lld)", fn, (long long)D);
@@ -341,9 +339,36 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
                                 "%s: bf16 strides must be multiples of 8 elements (16 bytes); operand %d "
                                 "has stride %lld",
                                 fn, a, (long long)st[a][x]);
+        if ((T + 127) / 128 * (B * H) > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+    } else {
+        if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: fp32 supports D <= 4096", fn);
+        if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
+            return fail(SWA_ERR_MISALIGNED, "%s: fp32 tensors must be 4-byte aligned", fn);
+        if ((B * H * T + swa::kSimtWarps - 1) / swa::kSimtWarps > INT32_MAX)
+            return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+    }
+    return SWA_OK;
+}
+
+}  // namespace swa_internal
+
+namespace {
+
+int forward_impl(const char* fn, const void* q, const void* k, const void* v, void* out, int64_t B,
+                 int64_t H, int64_t T, int64_t D, int64_t W, double scale, const int64_t* strides,
+                 int dtype, void* stream, float* lse = nullptr) {
+    int64_t st[4][3];
+    if (int rc = swa_internal::check_forward(fn, q, k, v, out, B, H, T, D, W, scale, strides, dtype, st))
+        return rc;
+    if (B == 0 || H == 0 || T == 0) return success();
+    const int Wi = (int)(W < T ? W : T);  // W >= T is causal attention
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+
+    if (dtype == SWA_BF16) {
         const int64_t BH = B * H;
         const int n_qt = (int)((T + 127) / 128);
-        if ((int64_t)n_qt * BH > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
         CUtensorMap mq, mk, mv;
         int rc;
         if ((rc = make_map(&mq, q, B, H, T, D, st[0])) || (rc = make_map(&mk, k, B, H, T, D, st[1])) ||
@@ -373,12 +398,8 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
                 mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
                 scale_log2, wait_limit(), ds->status);
     } else {
-        if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: fp32 supports D <= 4096", fn);
-        if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
-            return fail(SWA_ERR_MISALIGNED, "%s: fp32 tensors must be 4-byte aligned", fn);
         const int64_t nrows = B * H * T;
         const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;
-        if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
         const size_t smem = (size_t)swa::kSimtWarps * (2 * D + 32) * sizeof(float);
         swa::Strides sx;
         for (int x = 0; x < 3; ++x) {

@@ -98,3 +98,32 @@ def test_module_and_backward_errors(lib):
     assert lib.swa_forward_lse(p, p, p, p, p + 2, 1, 1, 16, 64, 4, 0.125, 1, None) == MISALIGNED
     assert b(p + 2, wb, 1, 1, 16, 64, 4, 0.125, 0, None) == MISALIGNED  # fp32 workspace 8
     assert b(p, wb, 0, 1, 16, 64, 4, 0.125, 1, None) == OK              # empty batch: no-op
+
+
+def test_forward_refusals_need_no_device(lib):
+    """Every refusal of the prefill, the dtype-specific ones included, is decided on the
+    host before the library asks the runtime for a device."""
+    p = DUMMY
+    f = lib.swa_forward
+    assert f(p, p, p, p, 1, 2, 8, 96, 4, 1, None) == UNSUPPORTED       # bf16 D = 96
+    assert f(p, p, p, p, 1, 2, 8, 5000, 4, 0, None) == UNSUPPORTED     # fp32 D > 4096
+    assert f(p + 8, p, p, p, 1, 2, 8, 64, 4, 1, None) == MISALIGNED    # bf16 16-byte rule
+    assert f(p + 2, p, p, p, 1, 2, 8, 64, 4, 0, None) == MISALIGNED    # fp32 4-byte rule
+    g = lib.swa_forward_ex
+    odd = strides(*([2 * 8 * 64, 8 * 64, 68] + [2 * 8 * 64, 8 * 64, 64] * 3))
+    assert g(p, p, p, p, 1, 2, 8, 64, 4, 0.125, odd, 1, None) == MISALIGNED
+    assert b"multiples of 8" in lib.swa_last_error()
+    assert g(p, p, p, p, 1, 2, 8, 64, 4, -1.0, None, 1, None) == UNSUPPORTED
+
+
+def test_module_refuses_before_its_first_gemm(lib):
+    """The module checks the attention's limits before it enqueues a projection: a
+    [B, T, H, Dh] stride T*d_model above 2^38 elements is refused as the attention would
+    refuse it, without the runtime being asked for a device."""
+    p = DUMMY
+    B, T, d, H = 1, 1 << 20, 1 << 19, 1 << 13
+    need = lib.swa_mha_workspace_bytes(B, T, d, 1)
+    assert need > 0
+    rc = lib.swa_mha_forward(p, p, None, p, None, p, None, p, None, p, p, need, B, T, d, H, 4, 1, None)
+    assert rc == INVALID
+    assert b"stride" in lib.swa_last_error()
