@@ -142,8 +142,10 @@ int swa_band_weights(const void* q, const void* k, float* weights,
  * keeps, growing it when a larger call needs more: make that first call before any
  * stream capture. Calls on one stream share its workspace; calls on different
  * streams do not.
- * Errors: as swa_forward; a negative pos[b] is found on the device: that stream's
- * output is written as zeros and swa_device_status() reports SWA_ERR_INVALID_ARG.
+ * Errors: as swa_forward, plus more than 65535 splits (possible only when SWA_DECODE_CHUNK
+ * forces a small chunk over a long ring) -> SWA_ERR_UNSUPPORTED. A negative pos[b] is found
+ * on the device: that stream's output is written as zeros and swa_device_status() reports
+ * SWA_ERR_INVALID_ARG.
  */
 int swa_decode(const void* q, const void* kring, const void* vring, const int64_t* pos,
                void* out, int64_t B, int64_t H, int64_t D, int64_t W, void* stream);

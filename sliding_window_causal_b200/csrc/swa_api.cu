@@ -277,6 +277,10 @@ int decode_workspace(void* stream, size_t part_need, size_t counters_need, float
     return SWA_OK;
 }
 
+// The splits are the grid's y dimension, whose limit is 65535 blocks. The library's own
+// plan stays below 148 * 16; only a small SWA_DECODE_CHUNK over a long ring can exceed it.
+constexpr int kMaxDecodeSplits = 65535;
+
 void split_plan(int64_t B, int64_t H, int64_t D, int64_t W, int32_t* splits, int32_t* chunk) {
     const int64_t rows_per_batch = (D == 64) ? swa::DecodeCfg<64>::kRowsPerBatch
                                              : swa::DecodeCfg<128>::kRowsPerBatch;
@@ -511,11 +515,14 @@ int swa_decode(const void* q, const void* kring, const void* vring, const int64_
         return fail(SWA_ERR_MISALIGNED, "swa_decode: tensors must be 16-byte aligned (pos 8-byte)");
     if (B * H > INT32_MAX || W > INT32_MAX / 2 || B * H > INT64_MAX / W / D)
         return fail(SWA_ERR_UNSUPPORTED, "swa_decode: sizes too large");
+    int32_t S, chunk;
+    split_plan(B, H, D, W, &S, &chunk);
+    if (S > kMaxDecodeSplits)
+        return fail(SWA_ERR_UNSUPPORTED, "swa_decode: %d splits exceed the grid limit of %d (a larger SWA_DECODE_CHUNK)",
+                    (int)S, kMaxDecodeSplits);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
-    int32_t S, chunk;
-    split_plan(B, H, D, W, &S, &chunk);
     float* part = nullptr;
     int* counters = nullptr;
     if (S > 1) {
@@ -842,6 +849,10 @@ extern "C" int swa_decode_noalloc(const void* q, const void* kring, const void* 
         return fail(SWA_ERR_UNSUPPORTED, "swa_decode_noalloc: sizes too large");
     int32_t S, chunk;
     split_plan(B, H, D, W, &S, &chunk);
+    if (S > kMaxDecodeSplits)
+        return fail(SWA_ERR_UNSUPPORTED,
+                    "swa_decode_noalloc: %d splits exceed the grid limit of %d (a larger SWA_DECODE_CHUNK)", (int)S,
+                    kMaxDecodeSplits);
     const size_t counter_bytes =
         ((size_t)(B * H) * sizeof(int) + kNoAllocCounterAlign - 1) / kNoAllocCounterAlign * kNoAllocCounterAlign;
     const size_t part_bytes = (size_t)(B * H) * S * (D + 2) * sizeof(float);

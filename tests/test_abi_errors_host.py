@@ -127,3 +127,18 @@ def test_module_refuses_before_its_first_gemm(lib):
     rc = lib.swa_mha_forward(p, p, None, p, None, p, None, p, None, p, p, need, B, T, d, H, 4, 1, None)
     assert rc == INVALID
     assert b"stride" in lib.swa_last_error()
+
+
+def test_decode_refuses_more_splits_than_the_grid_holds(lib, monkeypatch):
+    """A forced small chunk over a long ring would need more than 65535 splits (the grid's
+    y limit): refused before anything is enqueued. The library's own plan stays far below."""
+    from sliding_window_causal_b200 import split_plan
+    p = DUMMY
+    W = 1 << 24
+    assert split_plan(1, 1, 64, W)[0] <= 148 * 16
+    monkeypatch.setenv("SWA_DECODE_CHUNK", "1")
+    splits, chunk = split_plan(1, 1, 64, W)
+    assert splits > 65535 and splits * chunk >= W
+    for f in (lib.swa_decode, lib.swa_decode_noalloc):
+        assert f(p, p, p, p, p, 1, 1, 64, W, None) == UNSUPPORTED
+        assert b"65535" in lib.swa_last_error()
