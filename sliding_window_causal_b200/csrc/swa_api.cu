@@ -672,12 +672,14 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
         if (!aligned(workspace, 256) || !aligned(lse, 4))
             return fail(SWA_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned, lse 4-byte", fn);
         if (!(scale > 0.0)) return fail(SWA_ERR_UNSUPPORTED, "%s: the bf16 path needs scale > 0", fn);
-        DeviceState* ds;
-        if (int rc = device_state(&ds)) return rc;
         const int64_t BH = B * H;
         const int n_t = (int)((T + 127) / 128);
         const int64_t Tpad = (int64_t)n_t * 128;
-        if (BH * n_t > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+        // one CTA per (b, h, tile) in the products, one warp per padded row in the statistics
+        if (BH * n_t > INT32_MAX || (BH * Tpad + 7) / 8 > INT32_MAX)
+            return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+        DeviceState* ds;
+        if (int rc = device_state(&ds)) return rc;
         const int64_t cst[3] = {H * T * D, T * D, D};
         CUtensorMap mq, mk, mv, mdo;
         int rc;

@@ -142,3 +142,13 @@ def test_decode_refuses_more_splits_than_the_grid_holds(lib, monkeypatch):
     for f in (lib.swa_decode, lib.swa_decode_noalloc):
         assert f(p, p, p, p, p, 1, 1, 64, W, None) == UNSUPPORTED
         assert b"65535" in lib.swa_last_error()
+
+
+def test_backward_refuses_grids_it_cannot_launch(lib):
+    """Sizes whose statistics grid (one warp per padded row) would not fit a launch are
+    refused before the device is touched, not truncated."""
+    p = DUMMY
+    B, H, T = 1, 1 << 20, 1 << 15
+    wb = lib.swa_backward_workspace_bytes(B, H, T)
+    assert lib.swa_backward(p, p, p, p, p, p, p, p, p, p, wb, B, H, T, 64, 4, 0.125, 1, None) == UNSUPPORTED
+    assert b"too many tiles" in lib.swa_last_error()
