@@ -724,10 +724,10 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
     for (const void* p : ptrs)
         if (!aligned(p, esz)) return fail(SWA_ERR_MISALIGNED, "%s: tensors must be aligned to their element size", fn);
     if (!aligned(workspace, 8)) return fail(SWA_ERR_MISALIGNED, "%s: workspace must be 8-byte aligned", fn);
-    DeviceState* ds;
-    if (int rc = device_state(&ds)) return rc;
     const int64_t blocks = B * H * ((T + swa::kBwdRows - 1) / swa::kBwdRows);
     if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
     const int Wi = (int)(W < T ? W : T);
     const size_t smem = swa::bwd_smem_floats((int)D) * 4;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

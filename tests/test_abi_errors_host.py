@@ -152,3 +152,7 @@ def test_backward_refuses_grids_it_cannot_launch(lib):
     wb = lib.swa_backward_workspace_bytes(B, H, T)
     assert lib.swa_backward(p, p, p, p, p, p, p, p, p, p, wb, B, H, T, 64, 4, 0.125, 1, None) == UNSUPPORTED
     assert b"too many tiles" in lib.swa_last_error()
+    B, H, T = 1, 1 << 27, 1 << 7  # CUDA-core path: 2^31 row blocks
+    wb = lib.swa_backward_workspace_bytes(B, H, T)
+    assert lib.swa_backward(p, p, p, p, p, None, p, p, p, p, wb, B, H, T, 32, 4, 0.125, 0, None) == UNSUPPORTED
+    assert b"too many rows" in lib.swa_last_error()
