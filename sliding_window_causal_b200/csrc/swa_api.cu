@@ -479,11 +479,11 @@ int swa_band_weights(const void* q, const void* k, float* weights, int64_t B, in
         return fail(SWA_ERR_MISALIGNED, "%s: tensors must be aligned to their element size", fn);
     int64_t st[2][3];
     if (int rc = read_strides(fn, strides, 2, B, H, T, D, st)) return rc;
-    DeviceState* ds;
-    if (int rc = device_state(&ds)) return rc;
     const int64_t nrows = B * H * T;
     const int64_t blocks = (nrows + swa::kWeightWarps - 1) / swa::kWeightWarps;
     if (blocks > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many rows", fn);
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
     const size_t smem = (size_t)swa::kWeightWarps * D * sizeof(float);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == SWA_BF16)

@@ -55,6 +55,8 @@ def test_band_weights_errors(lib):
     assert f(p, p, None, 1, 2, 8, 64, 4, 0.1, None, 1, None) == INVALID
     assert f(p, p, p, 1, 2, 8, 64, 4, float("nan"), None, 1, None) == INVALID
     assert f(p, p, p, 1, 2, 8, 5000, 4, 0.1, None, 0, None) == UNSUPPORTED  # D > 4096
+    assert f(p, p, p, 1, 1 << 27, 1 << 7, 4, 1, 0.5, None, 0, None) == UNSUPPORTED  # 2^32 rows
+    assert b"too many rows" in lib.swa_last_error()
 
 
 def test_decode_and_streaming_errors(lib):
