@@ -54,6 +54,12 @@ MUTANTS = [
      [("dkh[j * D + d] += c * ds * qi[d];", "dkh[j * D + d] += ds * qi[d];")]),
     ("backward dv weighted by ds", [("dvh[j * D + d] += p[j - lo] * doi[d];", "dvh[j * D + d] += ds * doi[d];")]),
     ("weights unnormalised", [("wrow[j] = wrow[j] / denom;", "wrow[j] = wrow[j];")]),
+    ("backward dq built from query rows",
+     [("dqh[i * D + d] += c * ds * kh[j * D + d];", "dqh[i * D + d] += c * ds * qh[j * D + d];")]),
+    ("backward dp against k instead of v",
+     [("for (int64_t d = 0; d < D; ++d) dot += doi[d] * vh[j * D + d];",
+       "for (int64_t d = 0; d < D; ++d) dot += doi[d] * kh[j * D + d];")]),
+    ("backward dk built from dout", [("dkh[j * D + d] += c * ds * qi[d];", "dkh[j * D + d] += c * ds * doi[d];")]),
 ]
 
 _CHILD = r"""
@@ -89,3 +95,45 @@ def test_mutant_is_caught(name, edits):
         assert r.returncode == 0, f"mutant child crashed: {r.stderr[-2000:]}"
         failed = json.loads(r.stdout.strip().splitlines()[-1])
         assert failed, f"no pin caught mutant: {name}"
+
+
+# Mistakes planted in a copy of the module oracle's Python source (oracle.mha), on the
+# CPU; the copy replaces oracle.mha for the duration of the test only.
+PY_MUTANTS = [
+    ("module heads interleaved",
+     [("y.reshape(B, T, H, Dh).transpose(0, 2, 1, 3)", "y.reshape(B, T, Dh, H).transpose(0, 3, 1, 2)")]),
+    ("module bias dropped", [("return y if b is None else y + np.asarray(b, dtype=np.float64)", "return y")]),
+    ("module kernel transposed",
+     [("np.matmul(a, np.asarray(w, dtype=np.float64))", "np.matmul(a, np.asarray(w, dtype=np.float64).T)")]),
+    ("module output projection skipped", [("out = linear(concat, wo, bo)", "out = concat")]),
+    ("module heads concatenated in reverse order",
+     [("concat = o.transpose(0, 2, 1, 3)", "concat = o[:, ::-1].transpose(0, 2, 1, 3)")]),
+    ("module window one key wider", [("o = forward(q, k, v, W, lib=lib)", "o = forward(q, k, v, W + 1, lib=lib)")]),
+    ("module keys projected by the query kernel",
+     [("heads(linear(x, wk, bk))", "heads(linear(x, wq, bq))")]),
+]
+
+
+@pytest.mark.parametrize("name,edits", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_module_mutant_is_caught(name, edits, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    from oracle_pins import ALL_PINS
+
+    src = textwrap.dedent(inspect.getsource(oracle.mha))
+    for old, new in edits:
+        assert old in src, f"mutation anchor missing: {old}"
+        src = src.replace(old, new)
+    ns = dict(vars(oracle))
+    exec(compile(src, "<mutated oracle.mha>", "exec"), ns)
+    monkeypatch.setattr(oracle, "mha", ns["mha"])
+    lib = oracle._load()
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant: {name}"
