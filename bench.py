@@ -442,7 +442,9 @@ def main():
             "unit": "TFLOP/s", "ms_per_step": mms,
             "config": {"workload": f"mha module bf16 B{mB} T{mT} d{md} H{mH} W{mW}", "B": mB, "T": mT,
                        "d_model": md, "H": mH, "W": mW, "seed": 1006, "gemm_flops": gemm_flops,
-                       "band_flops": attn_flops},
+                       "band_flops": attn_flops,
+                       "l2": f"inputs larger than L2 (x {mB * mT * md * 2 / 2**20:.0f} MiB, kernels "
+                             f"{4 * md * md * 2 / 2**20:.0f} MiB), no flush"},
             "roofline": {"bound": "tensor", "achieved": mtf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": mtf / peak_tf, "peak_kind": f"{peak_kind} bf16 burst", "traffic": None},
             "clocks": mclk.summary(), "gpu_launches": args.steps,
@@ -467,12 +469,15 @@ def main():
             bms = timed(bstep, bsteps, stream, pg, device) / bsteps
         swa.device_status()
         bflops = 5 * band_flops(bw.B, bw.H, bw.T, bw.D, bw.W) // 2  # five band products
+        b_in = 5 * bw.B * bw.H * bw.T * bw.D * 2  # bytes of q, k, v, out, dout (bf16)
         btf = bflops / (bms * 1e-3) / 1e12
         backward_line = {
             "metric": "backward TFLOP/s (2.5 x band FLOPs)", "value": world * btf, "unit": "TFLOP/s",
             "ms_per_step": bms, "steps": bsteps,
             "config": {"workload": bw.name + " backward", "B": bw.B, "H": bw.H, "T": bw.T, "D": bw.D,
-                       "W": bw.W, "seed": bw.seed, "dout_seed": 1007, "useful_flops": bflops},
+                       "W": bw.W, "seed": bw.seed, "dout_seed": 1007, "useful_flops": bflops,
+                       "l2": f"inputs larger than L2 (q, k, v, out, dout {b_in / 2**20:.0f} MiB), no flush"
+                       if b_in > L2_BYTES else "inputs smaller than L2: L2-resident"},
             "roofline": {"bound": "tensor", "achieved": btf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": btf / peak_tf, "peak_kind": f"{peak_kind} bf16 burst", "traffic": None,
                          "products_issued_per_useful": 7 / 5},
