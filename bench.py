@@ -42,15 +42,27 @@ L2_BYTES = 126 * 2**20
 KERNEL_SOURCES = {"prefill": ["prefill_pp.cuh", "ptx.cuh", "umma.h", "plan.h"],
                   "decode": ["decode.cuh", "ptx.cuh"],
                   "chunk": ["chunk.cuh", "prefill_pp.cuh", "ptx.cuh", "umma.h", "plan.h"]}
+# Decode and chunk were captured with 16 of the 64 streams (1.07 GB of rings). Each stream
+# reads only its own ring, so traffic grows with the units processed (ring slots, chunk rows),
+# but the positions are random and 16 streams are not a quarter of them. The capture is
+# scaled by the kernel's algorithmic bytes, full workload over the 16-stream sample (the
+# chunk kernel's count leaves out the append's ring writes): (sample, full) below.
+SAMPLE_ALGORITHMIC_BYTES = {"decode": (951_025_792, 4_296_016_384),
+                            "chunk": (1_121_042_560, 4_508_746_240)}
+
+
+def _scaled(kind, captured):
+    sample, full = SAMPLE_ALGORITHMIC_BYTES[kind]
+    return captured * full / sample
+
+
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
     "prefill": {"bytes": 1135.2e6 + 112.2e6, "sources": "7b04bbdb520ca15e"},
-    # 16 of the 64 streams captured (1.07 GB of rings), scaled x4 by streams: each stream
-    # reads only its own ring, so traffic grows in proportion. decode.cuh is unchanged since
-    # the capture; ptx.cuh has since gained helpers the decode kernel does not use.
-    "decode": {"bytes": 4 * (951.0e6 + 3.5e6), "sources": "69ace3889ab1351e"},
-    # chunk_kernel, 16 of the 64 streams captured, scaled x4 by streams as for decode
-    "chunk": {"bytes": 4 * (1105.6e6 + 17.7e6), "sources": "d2e5b2317b60e3ce"},
+    # decode.cuh is unchanged since the capture; ptx.cuh has since gained helpers the
+    # decode kernel does not use
+    "decode": {"bytes": _scaled("decode", 951.0e6 + 3.5e6), "sources": "69ace3889ab1351e"},
+    "chunk": {"bytes": _scaled("chunk", 1105.6e6 + 17.7e6), "sources": "d2e5b2317b60e3ce"},
 }
 
 

@@ -3,12 +3,14 @@ brute-force enumeration of the band pairs."""
 import os
 import sys
 
+import pytest
 import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+from sliding_window_causal_b200 import inputs  # noqa: E402
 
 
 def brute_pairs(T, W):
@@ -60,3 +62,47 @@ def test_measured_traffic_matches_the_recorded_sources():
     for kind in bench.MEASURED_TRAFFIC:
         v = bench.measured_traffic(kind)
         assert v is None or v == bench.MEASURED_TRAFFIC[kind]["bytes"]
+
+
+def _skip_randn(gen, shape):
+    """Advance gen exactly as the input generator does for a tensor of this shape (the
+    same per-leading-index split), without keeping the numbers."""
+    n = 1
+    for s in shape:
+        n *= s
+    if n <= inputs.CHUNK or len(shape) == 1:
+        torch.randn(shape, generator=gen, dtype=torch.float32)
+        return
+    for _ in range(shape[0]):
+        _skip_randn(gen, shape[1:])
+
+
+def _positions(shapes, B, pos_max, seed):
+    gen = torch.Generator().manual_seed(seed)
+    for shp in shapes:
+        _skip_randn(gen, shp)
+    return torch.randint(0, pos_max, (B,), generator=gen, dtype=torch.int64)
+
+
+@pytest.mark.slow
+def test_sampled_traffic_is_scaled_by_the_workloads_algorithmic_bytes():
+    """The decode and chunk captures ran 16 of the 64 streams; the recorded (sample, full)
+    algorithmic byte counts that scale them are those of the seeded workloads."""
+    d, c = inputs.DECODE, inputs.CHUNKED
+    dshapes = lambda B: [(B, d.H, d.D), (B, d.H, d.W, d.D), (B, d.H, d.W, d.D)]
+    cshapes = lambda B: [(B, c.H, c.C, c.D)] * 3 + [(B, c.H, c.W, c.D)] * 2
+    # the walk reproduces the generator's positions
+    p16 = _positions(dshapes(16), 16, d.pos_max, d.seed)
+    assert torch.equal(p16, inputs.decode_inputs(16, d.H, d.D, d.W, d.pos_max, d.dtype, d.seed)[3])
+    q16 = _positions(cshapes(16), 16, c.pos_max, c.seed)
+    assert torch.equal(q16, inputs.chunk_inputs(16, c.H, c.C, c.D, c.W, c.pos_max, c.dtype, c.seed)[5])
+
+    got = {"decode": [], "chunk": []}
+    for B in (16, 64):
+        pd = _positions(dshapes(B), B, d.pos_max, d.seed)
+        got["decode"].append(bench.decode_bytes(B, d.H, d.D, d.W, pd))
+        pc = _positions(cshapes(B), B, c.pos_max, c.seed)
+        append_writes = B * c.H * min(c.C, c.W) * c.D * 2 * 2
+        got["chunk"].append(bench.chunk_work(B, c.H, c.C, c.D, c.W, pc)[1] - append_writes)
+    for kind in ("decode", "chunk"):
+        assert tuple(got[kind]) == bench.SAMPLE_ALGORITHMIC_BYTES[kind], kind
