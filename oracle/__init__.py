@@ -81,6 +81,11 @@ def forward(q, k, v, W, lib=None, scale=None):
     return out
 
 
+def max_threads(lib=None):
+    """Threads the oracle's parallel loops run with (OpenMP's team size)."""
+    return int((lib or _load()).swa_oracle_max_threads())
+
+
 def forward_rows(q, k, v, W, rows, lib=None):
     """Outputs [n, D] of the flattened query rows r = (b*H + h)*T + i listed in rows."""
     lib = lib or _load()

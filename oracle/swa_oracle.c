@@ -52,6 +52,7 @@
  * written.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -442,3 +443,7 @@ int swa_oracle_backward(const double* q, const double* k, const double* v, const
     }
     return bad ? ORACLE_INVALID : ORACLE_OK;
 }
+
+/* The number of threads an OpenMP parallel region of this library runs with: what the
+ * timings of these functions are reported against. */
+int swa_oracle_max_threads(void) { return omp_get_max_threads(); }

@@ -106,3 +106,19 @@ def test_sampled_traffic_is_scaled_by_the_workloads_algorithmic_bytes():
         got["chunk"].append(bench.chunk_work(B, c.H, c.C, c.D, c.W, pc)[1] - append_writes)
     for kind in ("decode", "chunk"):
         assert tuple(got[kind]) == bench.SAMPLE_ALGORITHMIC_BYTES[kind], kind
+
+
+def test_cpu_baseline_sample_is_described_as_taken():
+    """The CPU baseline reports the oracle's own thread count and a sample description that
+    matches the rows it ran, including when the sample wraps around the heads."""
+    import oracle
+    for wl, budget in ((inputs.SMALL, 0.3), (inputs.TINY[0], 0.05)):
+        q, k, v = inputs.for_workload(wl)
+        rate, desc, threads = bench.cpu_baseline_prefill(wl, budget, q, k, v)
+        assert rate > 0 and threads == oracle.max_threads()
+        rows = int(desc.split()[0])
+        assert rows > 0 and "in the oracle" in desc
+        if rows > wl.H * wl.T:
+            assert "round again" in desc
+        else:
+            assert "round again" not in desc
