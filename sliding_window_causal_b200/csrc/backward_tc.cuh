@@ -9,15 +9,15 @@
 //   bwd_stats_kernel  delta_i from dout and out, and lse_i (from the forward) in log2
 //                     units, into a [B*H, Tpad] layout padded to whole 128-row tiles
 //                     (padding rows get lse = +inf, delta = 0, so they weigh nothing).
-//   bwd_kv_kernel<D>  one CTA per (b, h, 128-key tile): K and V stay in shared memory;
+//   bwd_tc_kernel<D, true>: one CTA per (b, h, 128-key tile): K and V stay in shared memory;
 //                     for every query tile that meets the band, TMA brings Q, dO and the
 //                     tile's (lse, delta); S^T = K Q^T and dP^T = V dO^T go to TMEM; eight
-//                     warps (two per key row, 64 columns each) turn them into bf16 P^T and
+//                     warps (two threads per key row, 64 columns each) turn them into bf16 P^T and
 //                     dS^T over the dP^T columns; then dV += P^T dO and dK += dS^T Q
 //                     accumulate in TMEM (TS form: A from TMEM, B from shared memory). The
 //                     next tile's S^T is computed while the element-wise warps work: they
 //                     read their scores into registers first and release the S columns.
-//   bwd_q_kernel<D>   one CTA per (b, h, 128-query tile): Q and dO stay; for every key
+//   bwd_tc_kernel<D, false>: one CTA per (b, h, 128-query tile): Q and dO stay; for every key
 //                     tile of the band S = Q K^T and dP = dO V^T, then dS (bf16, in TMEM)
 //                     and dQ += dS K.
 // Work per band pair: seven 128x128xD products (the score and dP products are formed in
