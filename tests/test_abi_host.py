@@ -128,3 +128,54 @@ def test_workspace_sizes():
         assert lib.swa_mha_workspace_bytes(B, T, d, dt) == 4 * part + (32 << 20)
     assert lib.swa_mha_workspace_bytes(1, 5, 0, 1) == -1
     assert lib.swa_mha_workspace_bytes(1, 5, 8, 7) == -1
+
+
+def _c_prototypes():
+    """name -> (return type, [parameter types]) for every function swa.h declares."""
+    text = open(os.path.join(ROOT, "include", "swa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"([A-Za-z_][\w \*]*?)\b(swa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        types = []
+        if params and params != "void":
+            for p in params.split(","):
+                p = " ".join(p.split())
+                # drop the parameter name: the last identifier not part of the type
+                t = re.sub(r"\s*\b[A-Za-z_]\w*$", "", p) if not p.endswith("*") else p
+                types.append(t.replace(" *", "*").replace("const ", "").strip())
+        protos[name] = (ret.replace("const ", "").strip(), types)
+    return protos
+
+
+def _kind(ct):
+    """Class of a ctypes type as the C ABI sees it."""
+    import ctypes
+    if ct is None:
+        return "void"
+    if ct in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(ct, "_type_") and isinstance(ct._type_, type):
+        return "ptr"
+    return {ctypes.c_int64: "i64", ctypes.c_int32: "i32", ctypes.c_uint64: "u64",
+            ctypes.c_double: "f64"}[ct]
+
+
+def _c_kind(t):
+    if t.endswith("*"):
+        return "ptr"
+    return {"int64_t": "i64", "int": "i32", "uint64_t": "u64", "double": "f64", "void": "void"}[t]
+
+
+def test_ctypes_signatures_match_the_header():
+    """Every binding declares exactly the header's parameter list (count and ABI class of
+    each argument) and return type: a mismatch would pass arguments in the wrong
+    registers without any error."""
+    h = _native.lib()
+    protos = _c_prototypes()
+    assert set(protos) == set(_native.EXPORTS)
+    for name, (ret, params) in protos.items():
+        f = getattr(h, name)
+        assert f.argtypes is not None, name
+        got = [_kind(a) for a in f.argtypes]
+        want = [_c_kind(t) for t in params]
+        assert got == want, f"{name}: binding {got} vs header {want}"
+        assert _kind(f.restype) == _c_kind(ret), f"{name}: return {f.restype} vs {ret}"
