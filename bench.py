@@ -3,15 +3,18 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
 
 A step is one swa_forward over the Mistral-shaped workload (B=1, H=32, T=16384,
-D=128, W=4096, bf16), inputs resident in HBM. The same run then times swa_decode over
-the streaming workload (B=64 streams, H=32, D=128, W=4096 ring, positions uniform in
-[0, 100000)) in a second timed region and reports it under "decode", and the chunked
-streaming prefill (the same streams each taking 128 new tokens, swa_chunk_forward) in a
-third, under "chunk", and the multi-head module (cuBLASLt projections around the
-attention, B1 T16384 d_model 4096, 32 heads, W4096) in a fourth, under "module", and the
-backward of the Mistral-shaped prefill in a fifth, under "backward". Useful prefill FLOPs count the band only: 4*B*H*D*sum_i
-min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos; chunk bytes are
-the ring slots the chunk needs, its q, k, v, out, the appended rows and pos.
+D=128, W=4096, bf16), inputs resident in HBM. The same run then times, each in a timed
+region of its own: the window sweep (B=2, H=16, T=8192, D=128, W in {1, 256, 1024, 4096,
+8192}) under "sweep"; the small workload (B=1, H=8, T=512, D=64, W=128) with L2 hot and
+with L2 flushed between steps under "small"; swa_decode over the streaming workload (B=64
+streams, H=32, D=128, W=4096 ring, positions uniform in [0, 100000)) under "decode"; the
+chunked streaming prefill (the same streams each taking 128 new tokens,
+swa_chunk_forward) under "chunk"; the multi-head module (cuBLASLt projections around the
+attention, B1 T16384 d_model 4096, 32 heads, W4096) under "module"; and the backward of
+the Mistral-shaped prefill under "backward". Useful prefill FLOPs count the band only:
+4*B*H*D*sum_i min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos;
+chunk bytes are the ring slots the chunk needs, its q, k, v, out, the appended rows and
+pos.
 
 Under torchrun each rank runs the same workload on its own GPU (weak scaling, no
 collective on the data path); times are the max over ranks. `--impl reference` times
@@ -278,6 +281,61 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def roofline_point(F, nbytes, ms, peak_tf, peak_gbs, peak_kind):
+    """Roofline of one prefill launch: F band FLOPs and nbytes algorithmic bytes (q, k, v
+    read once, out written once) in ms. The bound is the tensor core when the arithmetic
+    intensity F / nbytes is at or above the ridge (peak FLOP/s over peak bytes/s), HBM
+    below it; `attainable` is min(tensor peak, intensity x HBM peak)."""
+    tf = F / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    ai = F / nbytes
+    ridge = peak_tf * 1e3 / peak_gbs
+    attainable = min(peak_tf, ai * peak_gbs / 1e3)
+    if ai >= ridge:
+        r = {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf}
+    else:
+        r = {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s", "frac": gbs / peak_gbs}
+    r.update({"peak_kind": peak_kind, "intensity_flop_per_byte": ai, "ridge_flop_per_byte": ridge,
+              "attainable_tflops": attainable, "frac_of_attainable": tf / attainable, "tflops": tf,
+              "gbs": gbs, "algorithmic_bytes": nbytes, "traffic": None})
+    return r
+
+
+def cpu_info():
+    """(CPU model name, logical CPU count) of this host."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+def cpu_one_thread_small(budget_s):
+    """The float64 oracle on the small workload (B1 H8 T512 D64 W128) on one thread, whole
+    calls repeated for about budget_s: (GFLOP/s, calls)."""
+    import oracle
+    wl = inputs.SMALL
+    q, k, v = (t.to(torch.float64).numpy() for t in inputs.for_workload(wl))
+    F = band_flops(wl.B, wl.H, wl.T, wl.D, wl.W)
+    n0 = oracle.max_threads()
+    oracle.set_threads(1)
+    try:
+        calls, t_or = 0, 0.0
+        while t_or < budget_s:
+            t1 = time.perf_counter()
+            oracle.forward(q, k, v, wl.W)
+            t_or += time.perf_counter() - t1
+            calls += 1
+    finally:
+        oracle.set_threads(n0)
+    return calls * F / t_or / 1e9, calls
+
+
 def prefill_workload(name):
     if name == "mistral":
         return inputs.MISTRAL
@@ -301,6 +359,8 @@ def main():
     ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--no-module", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-small", action="store_true")
     ap.add_argument("--backward-workload", default="mistral",
                     help="prefill workload whose backward the backward leg times (as --workload)")
     ap.add_argument("--chunk-streams", type=int, default=None,
@@ -364,6 +424,72 @@ def main():
                "h2d_bytes_per_step": 3 * qh.numel() * qh.element_size(),
                "d2h_bytes_per_step": outp.numel() * outp.element_size(), "steps": e2e_steps}
         del qp, kp, vp, outp
+
+    # ------------------------------------------------------------ window sweep
+    sweep = None
+    if not args.no_sweep:
+        sweep = []
+        for sw in inputs.SWEEP:
+            sq, sk, sv = (t.to(device) for t in inputs.for_workload(sw))
+            sout = torch.empty_like(sq)
+            sfn = lambda sq=sq, sk=sk, sv=sv, sout=sout, W=sw.W: swa.forward(sq, sk, sv, W, out=sout)
+            for _ in range(args.warmup):
+                sfn()
+            swa.device_status()
+            with ClockSampler(dev_index) as sclk:
+                sms = timed(sfn, args.steps, stream, pg, device) / args.steps
+            swa.device_status()
+            sF = band_flops(sw.B, sw.H, sw.T, sw.D, sw.W)
+            snb = 4 * sw.B * sw.H * sw.T * sw.D * 2
+            sweep.append({
+                "workload": sw.name, "W": sw.W, "band_flops": sF, "ms_per_step": sms,
+                "value": world * sF / (sms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "roofline": roofline_point(sF, snb, sms, peak_tf, peak_gbs, f"{peak_kind} bf16 burst / HBM copy"),
+                "l2": f"inputs larger than L2 (q, k, v {3 * sq.numel() * 2 / 2**20:.0f} MiB), no flush",
+                "clocks": sclk.summary(), "gpu_launches": args.steps, "seed": sw.seed})
+            del sq, sk, sv, sout, sfn
+        torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------ small workload (hot and cold L2)
+    small = None
+    if not args.no_small:
+        sw = inputs.SMALL
+        sq, sk, sv = (t.to(device) for t in inputs.for_workload(sw))
+        sout = torch.empty_like(sq)
+        sfn = lambda: swa.forward(sq, sk, sv, sw.W, out=sout)
+        for _ in range(args.warmup):
+            sfn()
+        swa.device_status()
+        with ClockSampler(dev_index) as hclk:
+            hot_ms = timed(sfn, args.steps, stream, pg, device) / args.steps
+        # cold L2: a 256 MiB buffer is written between steps, outside the timed events
+        flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=device)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        with ClockSampler(dev_index) as cclk2:
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                sfn()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+        cold_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, pg, device)
+        swa.device_status()
+        sF = band_flops(sw.B, sw.H, sw.T, sw.D, sw.W)
+        snb = 4 * sw.B * sw.H * sw.T * sw.D * 2
+        small = {
+            "workload": sw.name, "band_flops": sF, "seed": sw.seed,
+            "hot_l2": {"ms_per_step": hot_ms, "value": world * sF / (hot_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "l2": "inputs smaller than L2 (1.5 MiB): L2-resident between steps",
+                       "roofline": roofline_point(sF, snb, hot_ms, peak_tf, peak_gbs, f"{peak_kind} bf16 burst / HBM copy"),
+                       "clocks": hclk.summary()},
+            "cold_l2": {"ms_per_step": cold_ms, "value": world * sF / (cold_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                        "l2": "a 256 MiB buffer written between steps, outside the timed events",
+                        "roofline": roofline_point(sF, snb, cold_ms, peak_tf, peak_gbs, f"{peak_kind} bf16 burst / HBM copy"),
+                        "clocks": cclk2.summary()},
+            "gpu_launches": 2 * args.steps,
+            "note": "latency-bound: 32 query tiles (16 work items) on 148 SMs"}
+        del sq, sk, sv, sout, sfn, flush
+        torch.cuda.empty_cache()
 
     # ------------------------------------------------------------ decode
     decode_line = None
@@ -513,7 +639,12 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, desc, threads = cpu_baseline_prefill(wl, float(os.environ.get("SWA_CPU_BUDGET_S", "15")),
                                                   qh, kh, vh)
-        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+        model, ncpu = cpu_info()
+        one, calls = cpu_one_thread_small(2.0)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "cpu_model": model, "nproc": ncpu,
+               "one_thread": {"value": one, "unit": "GFLOP/s", "workload": inputs.SMALL.name,
+                              "sample": f"{calls} whole calls of the oracle on one thread"}}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -532,6 +663,8 @@ def main():
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
+        "sweep": sweep,
+        "small": small,
         "decode": decode_line,
         "chunk": chunk_line,
         "module": module_line,

@@ -86,6 +86,14 @@ def max_threads(lib=None):
     return int((lib or _load()).swa_oracle_max_threads())
 
 
+def set_threads(n, lib=None):
+    """Run the oracle's later parallel loops on n threads (OpenMP's team size)."""
+    lib = lib or _load()
+    lib.swa_oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.swa_oracle_set_threads.restype = None
+    lib.swa_oracle_set_threads(int(n))
+
+
 def forward_rows(q, k, v, W, rows, lib=None):
     """Outputs [n, D] of the flattened query rows r = (b*H + h)*T + i listed in rows."""
     lib = lib or _load()

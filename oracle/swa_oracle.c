@@ -447,3 +447,8 @@ int swa_oracle_backward(const double* q, const double* k, const double* v, const
 /* The number of threads an OpenMP parallel region of this library runs with: what the
  * timings of these functions are reported against. */
 int swa_oracle_max_threads(void) { return omp_get_max_threads(); }
+
+/* Team size of the parallel loops that follow (for timing the oracle on fewer threads). */
+void swa_oracle_set_threads(int n) {
+    if (n > 0) omp_set_num_threads(n);
+}
