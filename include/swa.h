@@ -101,6 +101,35 @@ int swa_forward_ex(const void* q, const void* k, const void* v, void* out,
                    double scale, const int64_t* strides, int dtype, void* stream);
 
 /*
+ * swa_forward_host: swa_forward from and to HOST memory, the copies overlapped with the
+ * attention and with each other.
+ *
+ *   q, k, v, out     : HOST [B,H,T,D] contiguous, of `dtype`. Page-locked (pinned) memory
+ *                      lets the copies run asynchronously and overlap; pageable memory
+ *                      works, but the copies then wait for each other.
+ *   dq, dk, dv, dout : DEVICE staging tensors of the same shape, owned by the caller; on
+ *                      return they hold the inputs and the output.
+ *   heads_per_group  : the (b,h) heads are independent problems (each row's band lies in
+ *                      its own head), so the B*H heads are processed in groups of this many
+ *                      consecutive heads; 0 lets the library pick (about eight groups).
+ * Group g's host-to-device copies, its attention (swa_forward on heads g) and its
+ * device-to-host copy run on three library-owned streams, created once per device and
+ * ordered by events, so the copies of one group overlap the attention of another and the
+ * two copy directions overlap each other. The work starts after everything already
+ * enqueued on `stream`, and `stream` waits for all of it: once the stream reaches this
+ * point, out holds the result, bitwise equal to swa_forward on the device copies. The
+ * copies are asynchronous: the host buffers must stay allocated and q, k, v unchanged
+ * until then. Calls from several host threads enqueue one after another.
+ * Errors: as swa_forward (on the device pointers), a null host pointer ->
+ * SWA_ERR_INVALID_ARG, heads_per_group < 0 -> SWA_ERR_INVALID_ARG. A CUDA failure after
+ * the first copy was enqueued returns SWA_ERR_CUDA with the earlier groups enqueued.
+ */
+int swa_forward_host(const void* q, const void* k, const void* v, void* out,
+                     void* dq, void* dk, void* dv, void* dout,
+                     int64_t B, int64_t H, int64_t T, int64_t D, int64_t W,
+                     int64_t heads_per_group, int dtype, void* stream);
+
+/*
  * swa_band_weights: the softmax weights of every query's band, for inspection.
  *
  * "Mistral Architecture > Implementation: Sliding Window Attention" (Step 2) returns the
@@ -338,6 +367,20 @@ int swa_decode_noalloc(const void* q, const void* kring, const void* vring, cons
  * qt*bm >= T).
  */
 int swa_prefill_tile_class(int64_t T, int64_t W, int64_t bm, int64_t bn, int64_t qt, int64_t kt);
+
+/*
+ * swa_prefill_work_item: the u-th work item of the tensor-core prefill (bf16, D 64 or
+ * 128) for sizes B, H, T and window W: the pair of 128-row query tiles (2*pair,
+ * 2*pair+1) of head (b, h). Items 0 .. B*H*ceil(ceil(T/128)/2) - 1 cover every pair
+ * once. First come the pairs of which both tiles exist and every row sees a whole
+ * window (256*pair >= min(W,T) - 1): all the same work, head after head, so that the
+ * CTAs at work together share a few heads' key and value tiles in L2. Then the lighter
+ * pairs, heaviest first, head-minor. The persistent CTAs take items in a snake order
+ * (CTA g of G: items g, 2G-1-g, 2G+g, ...). Writes *b, *h, *pair and returns 0, or
+ * returns -1 for invalid arguments (B, H, T or W < 1, u out of range, null pointers).
+ */
+int swa_prefill_work_item(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W, int64_t* b,
+                          int64_t* h, int64_t* pair);
 
 /*
  * swa_decode_valid_slots: number n of ring slots that hold in-window positions for a

@@ -292,22 +292,38 @@ def mha_forward(x, wq, bq, wk, bk, wv, bv, wo, bo, num_heads, window, out=None, 
     return out[0] if squeeze else out
 
 
-def forward_host(q, k, v, window, out=None, device=None, staging=None):
-    """Prefill from host tensors: copy q, k, v to the device on the current stream,
-    run forward, copy the result back into `out` (pinned host memory recommended).
-    `staging` may hold preallocated device tensors (q, k, v, out) to reuse."""
+def forward_host(q, k, v, window, out=None, device=None, staging=None, heads_per_group=0):
+    """Prefill from host tensors through swa_forward_host: q, k, v are contiguous
+    [B,H,T,D] CPU tensors (pinned memory lets the copies overlap); the result lands in
+    `out` (a CPU tensor, allocated pinned if None). The (b,h) heads are copied in, computed
+    and copied back in groups on the library's own streams, overlapped; the current
+    stream waits for all of it. `staging` may hold preallocated device tensors
+    (dq, dk, dv, dout) of the same shape. The copies are asynchronous: q, k, v and out
+    must stay alive (and unchanged) until the current stream has passed this call, e.g.
+    until a synchronize."""
     torch = _torch()
     device = torch.device(device or "cuda")
+    for t in (q, k, v):
+        if t.device.type != "cpu" or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must be contiguous CPU tensors of one shape and dtype")
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B,H,T,D]")
     if staging is None:
         staging = tuple(torch.empty(q.shape, dtype=q.dtype, device=device) for _ in range(4))
-    dq, dk, dv, dout = staging
-    dq.copy_(q, non_blocking=True)
-    dk.copy_(k, non_blocking=True)
-    dv.copy_(v, non_blocking=True)
-    forward(dq, dk, dv, window, out=dout)
+    _need_cuda(*staging)
+    if any(t.shape != q.shape or t.dtype != q.dtype for t in staging):
+        raise ValueError("staging tensors must match q's shape and dtype")
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    out.copy_(dout, non_blocking=True)
+    if out.device.type != "cpu" or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must be a contiguous CPU tensor like q")
+    B, H, T, D = q.shape
+    dq, dk, dv, dout = staging
+    with torch.cuda.device(device):
+        check(_native.lib().swa_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(),
+                                             B, H, T, D, int(window), int(heads_per_group), _dtype_code(q),
+                                             _stream_ptr(device)))
     return out
 
 
@@ -321,6 +337,14 @@ def device_status(stream=None):
 def tile_class(T, W, bm, bn, qt, kt):
     """0 not visited, 1 edge (masked), 2 full; -1 invalid. Host only, no GPU needed."""
     return _native.lib().swa_prefill_tile_class(T, W, bm, bn, qt, kt)
+
+
+def work_item(u, B, H, T, W):
+    """(b, h, pair) of the tensor-core prefill's u-th work item (see swa_prefill_work_item),
+    or None for invalid arguments."""
+    b, h, p = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    rc = _native.lib().swa_prefill_work_item(u, B, H, T, W, ctypes.byref(b), ctypes.byref(h), ctypes.byref(p))
+    return None if rc != 0 else (b.value, h.value, p.value)
 
 
 def valid_slots(pos, W):

@@ -10,9 +10,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_swa.so")
 
 # every exported symbol of include/swa.h
-EXPORTS = ("swa_forward", "swa_forward_ex", "swa_band_weights", "swa_decode", "swa_decode_noalloc",
+EXPORTS = ("swa_forward", "swa_forward_ex", "swa_forward_host", "swa_band_weights", "swa_decode", "swa_decode_noalloc",
            "swa_chunk_forward", "swa_ring_append", "swa_mha_forward", "swa_mha_workspace_bytes",
-           "swa_forward_lse", "swa_backward", "swa_backward_workspace_bytes", "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_decode_valid_slots", "swa_decode_split_plan",
+           "swa_forward_lse", "swa_backward", "swa_backward_workspace_bytes", "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_prefill_work_item", "swa_decode_valid_slots", "swa_decode_split_plan",
            "swa_set_wait_limit_ns", "swa_timeout_probe")
 
 SWA_F32, SWA_BF16 = 0, 1
@@ -44,6 +44,8 @@ def lib(path=None):
     h.swa_forward_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double,
                                  ctypes.POINTER(i64), i32, vp]
     h.swa_forward_ex.restype = i32
+    h.swa_forward_host.argtypes = [vp] * 8 + [i64] * 6 + [i32, vp]
+    h.swa_forward_host.restype = i32
     h.swa_band_weights.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double,
                                    ctypes.POINTER(i64), i32, vp]
     h.swa_band_weights.restype = i32
@@ -71,6 +73,9 @@ def lib(path=None):
     h.swa_last_error.restype = ctypes.c_char_p
     h.swa_prefill_tile_class.argtypes = [i64] * 6
     h.swa_prefill_tile_class.restype = i32
+    pi64 = ctypes.POINTER(i64)
+    h.swa_prefill_work_item.argtypes = [i64] * 5 + [pi64] * 3
+    h.swa_prefill_work_item.restype = i32
     h.swa_decode_valid_slots.argtypes = [i64, i64]
     h.swa_decode_valid_slots.restype = i64
     h.swa_decode_split_plan.argtypes = [i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int32),

@@ -35,6 +35,12 @@
 
 namespace swa {
 
+// mbar_wait for a whole warp: true only if every lane's wait completed, so that the warp
+// stays converged (its elected-lane MMAs need the full warp).
+__device__ __forceinline__ bool bwd_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, limit_ns, abort));
+}
+
 constexpr int kBwdTcThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2..9 element-wise
 constexpr int kBwdTcEw = 256;       // element-wise threads: two warps per row quarter
 
@@ -270,8 +276,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {
             // ---------------------------------------------------------------- MMA issuer
+            // (the whole warp runs this loop; its waits are warp-uniform, one lane issues)
             const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
             const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
             const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
@@ -281,14 +288,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const uint32_t fb_lo = ptx::smem_u32(smem + Cf::kFixOff + Cf::kTileBytes) >> 4;
             const uint32_t ring_lo = ptx::smem_u32(smem + Cf::kRingOff) >> 4;
             constexpr uint32_t kStageLo = Cf::kTileBytes >> 4;
-            bool ok = ptx::mbar_wait(fix_full, 0, wait_limit_ns, abort_flag);
+            bool ok = bwd_wait_warp(fix_full, 0, wait_limit_ns, abort_flag);
             auto next_visited = [&](int y) {  // the first visited tile after y (> hi if none)
                 for (++y; y <= hi && cls(y) == 0; ++y) {
                 }
                 return y;
             };
             auto wait_stage = [&](uint32_t idx) {
-                return ptx::mbar_wait(ring_full + idx % NS, (idx / NS) & 1, wait_limit_ns, abort_flag);
+                return bwd_wait_warp(ring_full + idx % NS, (idx / NS) & 1, wait_limit_ns, abort_flag);
             };
             // KV: S^T = K Q^T, dP^T = V dO^T.   Q: S = Q K^T, dP = dO V^T.
             // Tile j's streamed operands sit in stages L % NS (a: Q or K) and (L+1) % NS (b: dO or V).
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k), desc_hi | ((a_lo + off) | lo_k),
+                    ptx::mma_ss_one(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k), desc_hi | ((a_lo + off) | lo_k),
                                 idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
@@ -306,7 +313,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + Cf::kColDP, desc_hi | ((fb_lo + off) | lo_k), desc_hi | ((b_lo + off) | lo_k),
+                    ptx::mma_ss_one(tmem + Cf::kColDP, desc_hi | ((fb_lo + off) | lo_k), desc_hi | ((b_lo + off) | lo_k),
                                 idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
@@ -318,12 +325,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 ptx::tc_fence_after();
                 issue_s(0);
                 issue_dp(0);
-                ptx::tc_commit(s_full);
+                ptx::tc_commit_one(s_full);
             }
             while (ok) {
                 const int ynext = next_visited(yt);
                 // the next tile's scores as soon as this tile's S and dP are in registers
-                ok = ptx::mbar_wait(s_read, j & 1, wait_limit_ns, abort_flag);
+                ok = bwd_wait_warp(s_read, j & 1, wait_limit_ns, abort_flag);
                 if (ok && ynext <= hi) {
                     ok = wait_stage(L + 2);
                     if (ok) {
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                         issue_s(L + 2);
                     }
                 }
-                if (ok) ok = ptx::mbar_wait(p_full, j & 1, wait_limit_ns, abort_flag);
+                if (ok) ok = bwd_wait_warp(p_full, j & 1, wait_limit_ns, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint32_t sta = L % NS, stb = (L + 1) % NS;
@@ -341,34 +348,34 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     // dK += dS^T Q (A = dS^T, the first half; B = Q)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk) + 16,
+                        ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk) + 16,
                                     desc_hi | ((b_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
+                        ptx::mma_ts_one(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
                                     desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 } else {
                     // dQ += dS K (A = dS in the dP columns, B = K)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk),
+                        ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk),
                                     desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                ptx::tc_commit(ring_empty + sta);
-                ptx::tc_commit(ring_empty + stb);
+                ptx::tc_commit_one(ring_empty + sta);
+                ptx::tc_commit_one(ring_empty + stb);
                 if (ynext > hi) break;
                 // the next tile's dP, over this tile's P and dS, after the products above read them
                 ok = wait_stage(L + 3);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 issue_dp(L + 2);
-                ptx::tc_commit(s_full);
+                ptx::tc_commit_one(s_full);
                 L += 2;
                 ++j;
                 yt = ynext;
             }
-            if (ok) ptx::tc_commit(o_final);
-            if (!ok) {
+            if (ok) ptx::tc_commit_one(o_final);
+            if (!ok && lane == 0) {
                 atomicCAS(status, 0, 5);
                 *abort_flag = 1;
             }
@@ -482,8 +489,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 ptx::mbar_wait(stat_full + ss, (t / 2) & 1, kPPDrainLimitNs, nullptr);
             }
         }
-        if (warp == 1 && lane == 0) {
-            ptx::tc_commit(drain);
+        if (warp == 1) {
+            ptx::tc_commit_one(drain);
             ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
         }
         __syncthreads();

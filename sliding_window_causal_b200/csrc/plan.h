@@ -41,6 +41,57 @@ SWA_HD int tile_class(int64_t T, int64_t W, int64_t bm, int64_t bn, int64_t qt, 
     return full ? 2 : 1;
 }
 
+// Work items of the tensor-core prefill: pairs of query tiles (2p, 2p+1) of one (b,h),
+// n_pairs = ceil(n_qt / 2) per head, BH * n_pairs items in all. Item u is (bh, pair):
+//  - first the "full" pairs, both of whose tiles exist and every row of which sees a
+//    whole window (256p >= W - 1, so they all do the same work), head after head with
+//    the pairs of a head in order: the CTAs working at the same time then share the
+//    key and value tiles of a few heads, which stay in L2;
+//  - then the lighter pairs (rows near the start of a head, and a last pair that has
+//    only one tile), heaviest first and head-minor, so that the persistent CTAs, which
+//    take items in a snake order, finish together.
+// W is the window clamped to T. Returns false if u is out of range. I is the integer type
+// (int in the kernels, whose item counts fit 32 bits; int64_t on the host).
+template <typename I>
+SWA_HD bool prefill_item(I u, I BH, I n_qt, I W, I* bh, I* pair) {
+    const I n_pairs = (n_qt + 1) / 2;
+    if (u < 0 || BH < 1 || n_qt < 1 || u >= BH * n_pairs) return false;
+    const I full_end = n_qt / 2;  // pairs with both tiles
+    I pf0 = (W - 1 + 255) / 256;  // first pair whose rows all see W keys
+    if (pf0 > full_end) pf0 = full_end;
+    const I nf = full_end - pf0;
+    if (u < BH * nf) {
+        *bh = u / nf;
+        *pair = pf0 + u % nf;
+        return true;
+    }
+    const I v = u - BH * nf, idx = v / BH;
+    *bh = v % BH;
+    if (!(n_qt & 1)) {
+        *pair = pf0 - 1 - idx;  // pairs pf0-1 .. 0: their work falls with the pair index
+        return true;
+    }
+    // The last pair holds a single tile; it goes where its work falls among the others:
+    // after the pairs p* .. pf0-1 that do at least as much (binary search: the work of
+    // pair p, in 128-key tiles, is non-decreasing in p below pf0).
+    auto tiles = [&](I qt) {  // key tiles visited by query tile qt
+        const I lo = qt * 128 - W + 1;
+        return qt - (lo > 0 ? lo / 128 : 0) + 1;
+    };
+    const I wh = tiles(n_qt - 1);
+    I lo = 0, hi = pf0;  // smallest p in [0, pf0) with work(p) >= wh, or pf0
+    while (lo < hi) {
+        const I mid = (lo + hi) / 2;
+        if (tiles(2 * mid) + tiles(2 * mid + 1) >= wh) hi = mid;
+        else lo = mid + 1;
+    }
+    const I at = pf0 - lo;  // place of the single-tile pair in the list
+    if (idx < at) *pair = pf0 - 1 - idx;
+    else if (idx == at) *pair = n_pairs - 1;
+    else *pair = pf0 - idx;
+    return true;
+}
+
 SWA_HD int64_t decode_valid_slots(int64_t pos, int64_t W) {
     return pos + 1 < W ? pos + 1 : W;
 }

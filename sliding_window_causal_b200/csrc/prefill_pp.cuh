@@ -13,17 +13,21 @@
 // written with its own (b, h, t) strides.
 //
 // The grid holds at most one CTA per SM; CTA g takes items g, then 2G-1-g, then 2G+g, ...
-// of the list ordered heaviest first (a snake over the list), which balances the load
-// without any device-side queue.
+// (a snake over the list of prefill_item in plan.h: first the equal-work pairs head after
+// head, so that the CTAs at work share a few heads' key and value tiles in L2, then the
+// lighter pairs heaviest first), which balances the load without any device-side queue.
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0, lane 0     TMA producer: Q_A, Q_B per item, then K_kt and V_kt through one
 //                      NSTAGE-deep ring of 128-row tiles.
-//   warp 1             allocates the 512 TMEM columns; lane 0 issues every tcgen05 MMA in
-//                      the order PV_A(kt-1), S_A(kt), PV_B(kt-1), S_B(kt), so that the tensor
+//   warp 1             allocates the 512 TMEM columns; the warp runs the MMA loop and an
+//                      elected lane issues every tcgen05 MMA in the order PV_A(kt-1),
+//                      S_A(kt), PV_B(kt-1), S_B(kt), so that the tensor
 //                      core works on one tile's products while the other tile's softmax runs:
 //                        S_X = Q_X K^T   -> TMEM columns [128X, 128X+128)   (fp32)
 //                        O_X += P_X V    -> TMEM columns [256+128X, +D)     (fp32)
+//   warp 2             recomputes, in fp32 on the CUDA cores, the rows the softmax warps
+//                      found sharp (pp_fix_row), taking them from a queue in shared memory.
 //   warps 4..7 (A), 8..11 (B)   softmax of one query tile each, one row per thread (warp w
 //                      reads TMEM lanes 32*(w%4)..): running max and sum of the online
 //                      softmax ("Mistral Architecture > Implementation: Sliding Window
@@ -40,6 +44,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "plan.h"
 #include "ptx.cuh"
 #include "umma.h"
@@ -50,10 +56,10 @@ constexpr int kPPThreads = 384;
 // Register split (setmaxnreg): the CTA is launched with kPPLaunchRegs per thread
 // (384 x 168 = 64512); the producer/MMA warpgroup gives registers back down to
 // kPPRoleRegs and the two softmax warpgroups take them up to kPPSoftmaxRegs:
-// 128 x 96 + 256 x 200 = 63488 <= 64512. The host refuses to launch if the compiled kernel does
+// 128 x 104 + 256 x 200 = 64512. The host refuses to launch if the compiled kernel does
 // not use exactly kPPLaunchRegs (an increase the pool cannot cover would never return).
 constexpr int kPPLaunchRegs = 168;
-constexpr int kPPRoleRegs = 96;
+constexpr int kPPRoleRegs = 104;
 constexpr int kPPSoftmaxRegs = 200;
 static_assert(128 * kPPRoleRegs + 256 * kPPSoftmaxRegs <= kPPThreads * kPPLaunchRegs, "register split");
 constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow by 2^8 first
@@ -63,6 +69,29 @@ constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow
 // use up the error budget left by the output's own bf16 rounding.
 constexpr int kPPPreciseWindow = 32;
 constexpr uint64_t kPPDrainLimitNs = 200000000ull;
+// P of a tile is handed to the MMA issuer in this many parts (1, 2 or 4), so that the
+// first keys' P.V products run while the softmax still works on the last keys.
+constexpr int kPPParts = 4;
+static_assert(kPPParts == 1 || kPPParts == 2 || kPPParts == 4, "parts of a tile's P");
+// A row whose largest weight from a single-bf16-P tile ends up above kPPSharpShare of the
+// row's total weight, and one of whose outputs reaches kPPSharpOut in magnitude, is
+// recomputed in fp32 on the CUDA cores (pp_fix_row): such a key's bf16 rounding reaches
+// the output almost undamped, on top of the output's own bf16 rounding (2^-8 relative).
+constexpr float kPPSharpShare = 0.25f;
+constexpr float kPPSharpOut = 1.0f;
+// Sharp rows go through a queue in shared memory to warp 2 (otherwise idle), which
+// recomputes them while the softmax warps carry on; a full queue makes a softmax thread
+// wait for a free slot.
+constexpr int kPPFixSlots = 64;
+
+// Raw operand pointers and their (b, h, t) element strides, for the fp32 recomputation
+// of sharp rows (the tensor-core path reads q, k, v through tensor maps).
+struct PPRaw {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    int64_t sq[3], sk[3], sv[3];
+};
 
 template <int D>
 struct PPCfg {
@@ -73,11 +102,12 @@ struct PPCfg {
     static constexpr int kQOff = 0;                    // Q_A, Q_B
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-    // q_full[2], q_empty[2], ring_full[S], ring_empty[S], s_full[2], p_full[2],
+    // q_full[2], q_empty[2], ring_full[S], ring_empty[S], s_full[2], p_full[2][4],
     // o_final[2], o_free[2], drain
-    static constexpr int kNumBars = 4 + 2 * kStages + 9;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+    static constexpr int kNumBars = 4 + 2 * kStages + 15;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, 4 queue counters
+    static constexpr int kFixOff = (kMiscOff + 24 + 15) & ~15;  // queue of sharp rows: kPPFixSlots x 16 B
+    static constexpr int kSmemBytes = kFixOff + kPPFixSlots * 16 + 1024;  // + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     __device__ static constexpr uint32_t colS(int x) { return 128u * x; }
     __device__ static constexpr uint32_t colO(int x) { return 256u + 128u * x; }
@@ -96,9 +126,8 @@ struct PPItem {
 
 __device__ __forceinline__ PPItem pp_decode(int u, int BH, int H, int n_qt, int T, int W) {
     PPItem it;
-    const int n_pairs = (n_qt + 1) >> 1;
-    const int p = n_pairs - 1 - u / BH;  // heaviest pairs first
-    const int bh = u % BH;
+    int bh, p;
+    prefill_item<int>(u, BH, n_qt, W, &bh, &p);  // u is in range: pp_item checked it
     it.b = bh / H;
     it.h = bh - it.b * H;
     it.qt[0] = 2 * p;
@@ -117,6 +146,12 @@ __device__ __forceinline__ PPItem pp_decode(int u, int BH, int H, int n_qt, int 
     it.k0 = it.f[0];
     it.k1 = it.hasB ? it.l[1] : it.l[0];
     return it;
+}
+
+// mbar_wait for a whole warp: true only if every lane's wait completed, so that the warp
+// stays converged (its elected-lane MMAs need the full warp).
+__device__ __forceinline__ bool pp_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, limit_ns, abort));
 }
 
 __device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W <= kPPPreciseWindow; }
@@ -175,11 +210,19 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
 // normalised by the weights the MMAs multiply by.
 // MASK: 0 every key of the tile is in the row's band; 1 only columns cmin..cmax are; 2
 // columns cmin..cmax and cmin2..cmax2 are. before_rescale() runs (warp-uniformly) before O
-// is rescaled, for callers whose last P.V product may still be in flight.
-template <int D, int MASK, bool PRECISE, typename BeforeRescale>
-__device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
+// is rescaled, for callers whose last P.V product may still be in flight. after_part(s)
+// runs (warp-uniformly) once the stores of part s of P (keys 128s/kPPParts ..) have been
+// issued and the next chunk's arithmetic is done, so that the caller can hand that part
+// to the MMA issuer while the rest of the tile is computed.
+// Returns the row's largest scaled score in the tile (log2 units; -inf if none is in band).
+struct PPNoPart {
+    __device__ void operator()(int) const {}
+};
+
+template <int D, int MASK, bool PRECISE, typename BeforeRescale, typename AfterPart = PPNoPart>
+__device__ __forceinline__ float pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
                                         float& l, int cmin, int cmax, int cmin2, int cmax2,
-                                        BeforeRescale before_rescale) {
+                                        BeforeRescale before_rescale, AfterPart after_part = AfterPart()) {
     uint32_t v[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) ptx::tmem_ld32(scol + 32 * c, v[c]);
@@ -240,17 +283,145 @@ __device__ __forceinline__ void pp_tile(uint32_t scol, uint32_t ocol, float scal
             const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
             const float e0 = ptx::ex2(z.x), e1 = ptx::ex2(z.y);
             ph[t] = ptx::pack_bf16x2(e0, e1);
-            const ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
             if (PRECISE) {
+                const ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
                 pl[t] = ptx::pack_bf16x2(e0 - w.x, e1 - w.y);
                 acc[(t + 2) & 3] = ptx::add2(acc[(t + 2) & 3], {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
+                acc[t & 3] = ptx::add2(acc[t & 3], w);
+            } else {
+                acc[t & 3] = ptx::add_bf16x2_f32(ph[t], acc[t & 3]);
             }
-            acc[t & 3] = ptx::add2(acc[t & 3], w);
         }
+        // the previous part's stores have had this chunk's arithmetic to land
+        if (c > 0 && c % (4 / kPPParts) == 0) after_part(c / (4 / kPPParts) - 1);
         ptx::tmem_st16(scol + 32 * c, ph);
         if (PRECISE) ptx::tmem_st16(scol + 32 * c + 16, pl);
     }
+    after_part(kPPParts - 1);
     l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+    return tm;
+}
+
+__device__ __forceinline__ float pp_bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float pp_bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
+
+// Row i of head (b, h), recomputed by the whole warp in fp32 on the CUDA cores. The band
+// is taken 32 keys at a time: lane t scores key j0+t (fp32 FMA over d, ascending), the
+// chunk's maximum moves the running maximum, and each lane accumulates its D/32 output
+// columns over the chunk's keys in order. Loads are issued in batches ahead of their use
+// (128 bytes of a lane's key row; half a chunk of value columns at a time). The weights are
+// exact fp32 exponentials: no key's weight carries a bf16 rounding. Writes the bf16
+// output row and, when lse_out is not null, the natural log-sum-exp. Warp-collective; the
+// row has at least one key. Runs on the sharp-row worker warp, within that warpgroup's
+// register share.
+template <int D>
+__device__ __forceinline__ void pp_fix_row(const PPRaw& raw, int b, int h, int i, int W, float scale_log2,
+                                        __nv_bfloat16* orow, float* lse_out, int lane) {
+    constexpr int DPL = D / 32;  // output columns per lane: 4 (8 bytes) or 2 (4 bytes)
+    constexpr int NQ = D / 8;    // 16-byte pieces of a row
+    using VT = typename std::conditional<DPL == 4, uint2, uint32_t>::type;
+    const __nv_bfloat16* qrow = raw.q + b * raw.sq[0] + h * raw.sq[1] + (int64_t)i * raw.sq[2];
+    const __nv_bfloat16* kbase = raw.k + b * raw.sk[0] + h * raw.sk[1];
+    const __nv_bfloat16* vbase = raw.v + b * raw.sv[0] + h * raw.sv[1] + lane * DPL;
+    const int lo = i - W + 1 > 0 ? i - W + 1 : 0;
+    float m = -INFINITY, lsum = 0.f, o[DPL];
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) o[c] = 0.f;
+    for (int j0 = lo; j0 <= i; j0 += 32) {
+        const int j = j0 + lane;
+        const bool mine = j <= i;
+        const __nv_bfloat16* krow = kbase + (int64_t)(mine ? j : i) * raw.sk[2];
+        VT vv[16];
+        auto load_v = [&](int t0) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const int jt = j0 + t0 + t <= i ? j0 + t0 + t : i;  // rows past i are never read
+                vv[t] = *reinterpret_cast<const VT*>(vbase + (int64_t)jt * raw.sv[2]);
+            }
+        };
+        load_v(0);
+        float acc = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < NQ; c0 += 8) {  // the key row in pieces of 128 bytes
+            uint4 kv[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) kv[c] = *reinterpret_cast<const uint4*>(krow + 8 * (c0 + c));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 qc = *reinterpret_cast<const uint4*>(qrow + 8 * (c0 + c));  // the same for every lane
+                const uint32_t qw[4] = {qc.x, qc.y, qc.z, qc.w};
+                const uint32_t kw[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc = fmaf(pp_bf16_lo(qw[e]), pp_bf16_lo(kw[e]), acc);
+                    acc = fmaf(pp_bf16_hi(qw[e]), pp_bf16_hi(kw[e]), acc);
+                }
+            }
+        }
+        const float s = mine ? acc * scale_log2 : -INFINITY;
+        float cm = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+        if (cm > m) {  // warp-uniform: the chunk raises the running maximum
+            const float a = exp2f(m - cm);  // 0 on the first chunk
+            lsum *= a;
+#pragma unroll
+            for (int c = 0; c < DPL; ++c) o[c] *= a;
+            m = cm;
+        }
+        const float p = mine ? exp2f(s - m) : 0.f;
+        lsum += p;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            if (half == 1) load_v(16);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const float pt = __shfl_sync(0xffffffffu, p, 16 * half + t);  // 0 for keys past i
+                if constexpr (DPL == 4) {
+                    o[0] = fmaf(pt, pp_bf16_lo(vv[t].x), o[0]);
+                    o[1] = fmaf(pt, pp_bf16_hi(vv[t].x), o[1]);
+                    o[2] = fmaf(pt, pp_bf16_lo(vv[t].y), o[2]);
+                    o[3] = fmaf(pt, pp_bf16_hi(vv[t].y), o[3]);
+                } else {
+                    o[0] = fmaf(pt, pp_bf16_lo(vv[t]), o[0]);
+                    o[1] = fmaf(pt, pp_bf16_hi(vv[t]), o[1]);
+                }
+            }
+        }
+    }
+    float l = lsum;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    const float inv = 1.f / l;
+    if constexpr (DPL == 4) {
+        uint2 w;
+        w.x = ptx::pack_bf16x2(o[0] * inv, o[1] * inv);
+        w.y = ptx::pack_bf16x2(o[2] * inv, o[3] * inv);
+        *reinterpret_cast<uint2*>(orow + lane * DPL) = w;
+    } else {
+        *reinterpret_cast<uint32_t*>(orow + lane * DPL) = ptx::pack_bf16x2(o[0] * inv, o[1] * inv);
+    }
+    if (lse_out != nullptr && lane == 0) *lse_out = (m + log2f(l)) * 0.6931471805599453f;
+}
+
+// Push row i of head (b, h) to the sharp-row queue: take the next push number s, wait
+// (bounded) until the worker has finished push s - kPPFixSlots, whose slot this is, write
+// the row, then its sequence word s + 1. Returns false on abort or time-out.
+__device__ __forceinline__ bool pp_push_sharp(uint32_t* fix_head, const uint32_t* fix_tail, uint4* fix_slot, int b,
+                                              int h, int i, uint64_t limit_ns, volatile int* abort) {
+    const uint32_t sl = atomicAdd(fix_head, 1u);
+    volatile uint4* e = fix_slot + (sl % kPPFixSlots);
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (*reinterpret_cast<const volatile uint32_t*>(fix_tail) + kPPFixSlots <= sl) {
+        if (*abort || ptx::globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(256);
+    }
+    e->x = (uint32_t)b;
+    e->y = (uint32_t)h;
+    e->z = (uint32_t)i;
+    __threadfence_block();
+    e->w = sl + 1;
+    return true;
 }
 
 // LSE: also write the natural log-sum-exp of each row (a separate instantiation, so that
@@ -261,7 +432,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                       int64_t osb, int64_t osh, int64_t ost, float* __restrict__ lse, int BH, int H,
                       int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
-                      int* status) {
+                      int* status, const __grid_constant__ PPRaw raw) {
     using C = PPCfg<D>;
     constexpr int NS = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -273,12 +444,20 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     uint64_t* ring_full = bars + 4;     // [NS]
     uint64_t* ring_empty = ring_full + NS;
     uint64_t* s_full = ring_empty + NS;  // [2]
-    uint64_t* p_full = s_full + 2;       // [2]
-    uint64_t* o_final = p_full + 2;      // [2]
+    uint64_t* p_full = s_full + 2;       // [2][4]: P of tile x, part s, is in TMEM
+    uint64_t* o_final = p_full + 8;      // [2]
     uint64_t* o_free = o_final + 2;      // [2]
     uint64_t* drain = o_free + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+    // queue of sharp rows: fix_head counts the rows pushed, fix_tail the rows the worker has
+    // finished, fix_done the softmax warps that finished, fix_beat their items (progress);
+    // push number s sits in slot s % kPPFixSlots as (b, h, i, s + 1)
+    uint32_t* fix_head = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 8);
+    uint32_t* fix_done = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 12);
+    uint32_t* fix_beat = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 16);
+    uint32_t* fix_tail = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 20);
+    uint4* fix_slot = reinterpret_cast<uint4*>(smem + C::kFixOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = ((n_qt + 1) >> 1) * BH;
@@ -289,7 +468,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             ptx::mbar_init(q_full + x, 1);
             ptx::mbar_init(q_empty + x, 1);
             ptx::mbar_init(s_full + x, 1);
-            ptx::mbar_init(p_full + x, 128);
+            for (int c = 0; c < 4; ++c) ptx::mbar_init(p_full + 4 * x + c, 4);  // one arrival per warp
             ptx::mbar_init(o_final + x, 1);
             ptx::mbar_init(o_free + x, 128);
         }
@@ -299,6 +478,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
+        *fix_head = 0;
+        *fix_done = 0;
+        *fix_beat = 0;
+        *fix_tail = 0;
+        for (int q = 0; q < kPPFixSlots; ++q) fix_slot[q] = make_uint4(0, 0, 0, 0);
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -360,8 +544,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {
             // ------------------------------------------------------------ MMA issuer
+            // (the whole warp runs this loop; its waits are warp-uniform, one lane issues)
             // Descriptors: the high word (SBO = 1024, sm_100 version, 128-byte swizzle) is
             // the same for every operand; the low word is start >> 4 plus the leading byte
             // offset field, so each MMA needs one add (shared memory is far below 256 KiB, so
@@ -387,7 +572,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (x < nx && ok) ok = ptx::mbar_wait(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
+                    if (x < nx && ok) ok = pp_wait_warp(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
                 }
                 if (!ok) break;
                 int pend[2] = {-1, -1};
@@ -397,8 +582,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     const uint32_t j = (uint32_t)(kt - it.k0);
                     const uint32_t Lk = Lbase + 2 * j, Lv = Lk - 1;
                     const uint32_t stk = Lk % NS, stv = Lv % NS;
-                    if (kt <= it.k1) ok = ptx::mbar_wait(ring_full + stk, (Lk / NS) & 1, wait_limit_ns, abort_flag);
-                    if (ok && kt > it.k0) ok = ptx::mbar_wait(ring_full + stv, (Lv / NS) & 1, wait_limit_ns, abort_flag);
+                    if (kt <= it.k1) ok = pp_wait_warp(ring_full + stk, (Lk / NS) & 1, wait_limit_ns, abort_flag);
+                    if (ok && kt > it.k0) ok = pp_wait_warp(ring_full + stv, (Lv / NS) & 1, wait_limit_ns, abort_flag);
                     if (!ok) break;
                     const uint32_t k_lo = (ring_lo + stk * kStageLo) | lo_k;
                     const uint32_t v_lo = (ring_lo + stv * kStageLo) | lo_v;
@@ -406,25 +591,31 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     for (int x = 0; x < 2; ++x) {
                         if (x >= nx || !ok) break;
                         if (pend[x] >= 0) {
-                            // PV_x(kt-1): needs P_x(kt-1), and O_x free if it starts the item
-                            ok = ptx::mbar_wait(p_full + x, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
-                            if (ok && first_pv[x] && ni[x] > 0)
-                                ok = ptx::mbar_wait(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
-                            if (!ok) break;
-                            ptx::tc_fence_after();
+                            // PV_x(kt-1) part by part as the softmax hands P_x(kt-1) over; O_x
+                            // must be free if it starts the item
+                            if (first_pv[x] && ni[x] > 0)
+                                ok = pp_wait_warp(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
-                                            desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
-                                            (!first_pv[x] || kk > 0) ? 1u : 0u);
-                            if (prec[x]) {
+                            for (int part = 0; part < kPPParts && ok; ++part) {
+                                ok = pp_wait_warp(p_full + 4 * x + part, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
+                                if (!ok) break;
+                                ptx::tc_fence_after();
+                                constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
 #pragma unroll
-                                for (int kk = 0; kk < 8; ++kk)
-                                    ptx::mma_ts(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
-                                                desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u);
+                                for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                    ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
+                                                    desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
+                                                    (!first_pv[x] || kk > 0) ? 1u : 0u);
+                                if (prec[x]) {
+#pragma unroll
+                                    for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                        ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                        desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u);
+                                }
                             }
+                            if (!ok) break;
                             first_pv[x] = false;
-                            if (pend[x] == it.l[x]) ptx::tc_commit(o_final + x);
+                            if (pend[x] == it.l[x]) ptx::tc_commit_one(o_final + x);
                             pend[x] = -1;
                         } else {
                             ptx::tc_fence_after();
@@ -434,27 +625,68 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                                ptx::mma_ss(tmem + C::colS(x), desc_hi | (q_lo[x] + off), desc_hi | (k_lo + off),
+                                ptx::mma_ss_one(tmem + C::colS(x), desc_hi | (q_lo[x] + off), desc_hi | (k_lo + off),
                                             idesc_s, kk > 0 ? 1u : 0u);
                             }
-                            ptx::tc_commit(s_full + x);
+                            ptx::tc_commit_one(s_full + x);
                             ++ns[x];
-                            if (kt == it.l[x]) ptx::tc_commit(q_empty + x);
+                            if (kt == it.l[x]) ptx::tc_commit_one(q_empty + x);
                             pend[x] = kt;
                         }
                     }
                     if (!ok) break;
-                    if (kt <= it.k1) ptx::tc_commit(ring_empty + stk);  // K(kt) read by its S MMAs
-                    if (kt > it.k0) ptx::tc_commit(ring_empty + stv);   // V(kt-1) read by its PV MMAs
+                    if (kt <= it.k1) ptx::tc_commit_one(ring_empty + stk);  // K(kt) read by its S MMAs
+                    if (kt > it.k0) ptx::tc_commit_one(ring_empty + stv);   // V(kt-1) read by its PV MMAs
                 }
                 L = Lbase + 2u * (uint32_t)(it.k1 - it.k0 + 1);
                 ++ni[0];
                 if (it.hasB) ++ni[1];
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 atomicCAS(status, 0, 5);
                 *abort_flag = 1;
             }
+        }
+      } else if (warp == 2) {
+        // ------------------------------------------------------------ sharp-row worker
+        // Slots are taken in push order. The loop ends once every softmax warp has
+        // finished and no push is left, or on abort, or when the softmax warps have made
+        // no progress (no item finished, nothing pushed) for the wait limit.
+        uint64_t t0 = ptx::globaltimer_ns();
+        uint32_t seen = 0;
+        for (uint32_t sl = 0;; ++sl) {
+            volatile uint4* e = fix_slot + (sl % kPPFixSlots);
+            bool have = false;
+            while (true) {
+                const uint32_t now = *reinterpret_cast<volatile uint32_t*>(fix_beat) +
+                                     *reinterpret_cast<volatile uint32_t*>(fix_head);
+                if (now != seen) {
+                    seen = now;
+                    t0 = ptx::globaltimer_ns();
+                }
+                if (e->w == sl + 1) {
+                    have = true;
+                    break;
+                }
+                if (*reinterpret_cast<volatile uint32_t*>(fix_done) == 8u &&
+                    *reinterpret_cast<volatile uint32_t*>(fix_head) <= sl)
+                    break;  // all softmax warps are done and nothing more was pushed
+                if (*abort_flag) break;
+                if (ptx::globaltimer_ns() - t0 > wait_limit_ns) {
+                    atomicCAS(status, 0, 5);
+                    *abort_flag = 1;
+                    break;
+                }
+                __nanosleep(256);
+            }
+            if (!__all_sync(0xffffffffu, have)) break;
+            __threadfence_block();
+            const uint4 ent = *const_cast<const uint4*>(reinterpret_cast<volatile uint4*>(e));
+            const int fb = (int)ent.x, fh = (int)ent.y, fi = (int)ent.z;
+            pp_fix_row<D>(raw, fb, fh, fi, W, scale_log2, out + fb * osb + fh * osh + (int64_t)fi * ost,
+                          LSE ? lse + ((int64_t)fb * H + fh) * T + fi : nullptr, lane);
+            __syncwarp();
+            if (lane == 0) *reinterpret_cast<volatile uint32_t*>(fix_tail) = sl + 1;  // slot free again
         }
       }
     } else {
@@ -481,6 +713,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             if (lo < 0) lo = 0;
             const int hi = i < T - 1 ? i : T - 1;
             float m_ref = -INFINITY, l = 0.f;
+            float t_np = -INFINITY;  // largest scaled score met in a single-bf16-P tile
             for (int kt = fx; kt <= lx; ++kt) {
                 bool w = ptx::mbar_wait(s_full + x, ns & 1, wait_limit_ns, abort_flag);
                 ++ns;
@@ -491,16 +724,20 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const uint32_t scol = tl + C::colS(x), ocol = tl + C::colO(x);
                 // S_x(kt) complete implies PV_x(kt-1) complete: nothing to wait for
                 const auto none = [] {};
+                // part s of P is in TMEM: the warp's stores have completed
+                const auto hand = [&](int part) {
+                    ptx::tmem_st_wait();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(p_full + 4 * x + part);
+                };
                 if (edge) {
-                    if (precise) pp_tile<D, 1, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
-                    else pp_tile<D, 1, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
+                    if (precise) pp_tile<D, 1, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand);
+                    else t_np = fmaxf(t_np, pp_tile<D, 1, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand));
                 } else {
-                    if (precise) pp_tile<D, 0, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
-                    else pp_tile<D, 0, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none);
+                    if (precise) pp_tile<D, 0, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand);
+                    else t_np = fmaxf(t_np, pp_tile<D, 0, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand));
                 }
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(p_full + x);
             }
             if (!ok) break;
             // ------------------------------------------------------------ epilogue
@@ -509,30 +746,67 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             ptx::tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            // natural log-sum-exp of the row's scaled scores: (m + log2 l) ln 2
-            if (LSE && i < T) lse[((int64_t)it.b * H + it.h) * T + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
             __nv_bfloat16* orow = out + it.b * osb + it.h * osh + (int64_t)i * ost;
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
-                ptx::tmem_ld_wait();
-                ptx::reg_fence(o);
-                if (i < T) {
+            const auto store_chunk = [&](int cc, const uint32_t (&o)[32]) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        uint4 val;
-                        val.x = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 0]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l);
-                        val.y = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l);
-                        val.z = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l);
-                        val.w = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l);
-                        *reinterpret_cast<uint4*>(orow + cc * 32 + t * 8) = val;
-                    }
+                for (int t = 0; t < 4; ++t) {
+                    uint4 val;
+                    val.x = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 0]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l);
+                    val.y = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l);
+                    val.z = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l);
+                    val.w = ptx::pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l);
+                    *reinterpret_cast<uint4*>(orow + cc * 32 + t * 8) = val;
+                }
+            };
+            // A row is sharp when one key of a single-bf16-P tile holds more than
+            // kPPSharpShare of its weight (t_np and m_ref are both log2 units; l is in the
+            // frame of m_ref) and some output reaches kPPSharpOut in magnitude, where the
+            // output's own bf16 spacing leaves little of the error budget to the weights. A
+            // sharp row is recomputed by the worker instead of stored from O.
+            const bool dominated = i < T && t_np != -INFINITY && ptx::ex2(t_np - m_ref) > kPPSharpShare * l;
+            bool sharp = false;
+            if (__any_sync(0xffffffffu, dominated)) {
+                // rare: the whole row of O first, to see its largest output
+                uint32_t o[D / 32][32];
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o[cc]);
+                ptx::tmem_ld_wait();
+                float big = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    ptx::reg_fence(o[cc]);
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) big = fmaxf(big, fabsf(__uint_as_float(o[cc][t])));
+                }
+                sharp = dominated && big * inv_l >= kPPSharpOut;
+                if (i < T && !sharp) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) store_chunk(cc, o[cc]);
+                }
+            } else {
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(tl + C::colO(x) + cc * 32, o);
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(o);
+                    if (i < T) store_chunk(cc, o);
                 }
             }
+            // natural log-sum-exp of the row's scaled scores: (m + log2 l) ln 2
+            if (LSE && i < T && !sharp)
+                lse[((int64_t)it.b * H + it.h) * T + i] = (m_ref + log2f(l)) * 0.6931471805599453f;
             ptx::tc_fence_before();
             ptx::mbar_arrive(o_free + x);  // O_x may be overwritten by the next item
+            if (sharp && !pp_push_sharp(fix_head, fix_tail, fix_slot, it.b, it.h, i, wait_limit_ns, abort_flag)) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+            if (lane == 0) atomicAdd(fix_beat, 1u);  // progress, for the worker's time limit
         }
+        __syncwarp();
+        __threadfence_block();  // this warp's pushes are visible before it counts as done
+        if (lane == 0) atomicAdd(fix_done, 1u);
         if (!ok) {
             atomicCAS(status, 0, 5);
             *abort_flag = 1;
@@ -553,8 +827,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);
             }
         }
-        if (warp == 1 && lane == 0) {
-            ptx::tc_commit(drain);  // completes when every MMA issued so far is done
+        if (warp == 1) {
+            ptx::tc_commit_one(drain);  // completes when every MMA issued so far is done
             ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
         }
         __syncthreads();

@@ -13,6 +13,7 @@
 #include <mutex>
 #include <string>
 #include <utility>
+#include <vector>
 
 #include "swa.h"
 #include "api_internal.h"
@@ -385,22 +386,31 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
         const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
         const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
         auto* ob = static_cast<__nv_bfloat16*>(out);
+        swa::PPRaw raw;
+        raw.q = static_cast<const __nv_bfloat16*>(q);
+        raw.k = static_cast<const __nv_bfloat16*>(k);
+        raw.v = static_cast<const __nv_bfloat16*>(v);
+        for (int x = 0; x < 3; ++x) {
+            raw.sq[x] = st[0][x];
+            raw.sk[x] = st[1][x];
+            raw.sv[x] = st[2][x];
+        }
         if (D == 128 && lse)
             swa::prefill_pp_kernel<128, true><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
                 mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status);
+                scale_log2, wait_limit(), ds->status, raw);
         else if (D == 128)
             swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
                 mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status);
+                scale_log2, wait_limit(), ds->status, raw);
         else if (lse)
             swa::prefill_pp_kernel<64, true><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
                 mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status);
+                scale_log2, wait_limit(), ds->status, raw);
         else
             swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
                 mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status);
+                scale_log2, wait_limit(), ds->status, raw);
     } else {
         const int64_t nrows = B * H * T;
         const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;
@@ -421,6 +431,37 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
     return success();
 }
 
+// ------------------------------------------------------------------ host-buffer pipeline
+// Per device: the three streams of swa_forward_host (host-to-device copies, attention,
+// device-to-host copies) and a pool of events that order them. Created on first use and
+// kept until exit. A call holds `mu` while it enqueues, so calls from several host
+// threads take the streams one after another.
+struct HostPipe {
+    std::mutex mu;
+    cudaStream_t in = nullptr, cmp = nullptr, out = nullptr;
+    std::vector<cudaEvent_t> ev;
+};
+std::map<int, HostPipe> g_pipe;
+
+HostPipe& host_pipe(int dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_pipe[dev];
+}
+
+// Streams and at least n_events events; the caller holds hp.mu.
+int host_pipe_ready(HostPipe& hp, size_t n_events) {
+    cudaError_t e = cudaSuccess;
+    for (cudaStream_t* st : {&hp.in, &hp.cmp, &hp.out})
+        if (!*st && e == cudaSuccess) e = cudaStreamCreateWithFlags(st, cudaStreamNonBlocking);
+    while (e == cudaSuccess && hp.ev.size() < n_events) {
+        cudaEvent_t x;
+        e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+        if (e == cudaSuccess) hp.ev.push_back(x);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "swa_forward_host: stream/event creation");
+    return SWA_OK;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -437,6 +478,17 @@ uint64_t swa_set_wait_limit_ns(uint64_t ns) {
 int swa_prefill_tile_class(int64_t T, int64_t W, int64_t bm, int64_t bn, int64_t qt, int64_t kt) {
     if (T < 1 || W < 1 || bm < 1 || bn < 1 || qt < 0 || kt < 0 || qt * bm >= T) return -1;
     return swa::tile_class(T, W, bm, bn, qt, kt);
+}
+
+int swa_prefill_work_item(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W, int64_t* b, int64_t* h,
+                          int64_t* pair) {
+    if (B < 1 || H < 1 || T < 1 || W < 1 || !b || !h || !pair || B > INT32_MAX || H > INT32_MAX || T > INT32_MAX)
+        return -1;
+    int64_t bh;
+    if (!swa::prefill_item<int64_t>(u, B * H, (T + 127) / 128, W < T ? W : T, &bh, pair)) return -1;
+    *b = bh / H;
+    *h = bh % H;
+    return 0;
 }
 
 int64_t swa_decode_valid_slots(int64_t pos, int64_t W) {
@@ -456,6 +508,61 @@ int swa_forward(const void* q, const void* k, const void* v, void* out, int64_t 
                 int64_t T, int64_t D, int64_t W, int dtype, void* stream) {
     return forward_impl("swa_forward", q, k, v, out, B, H, T, D, W,
                         D >= 1 ? 1.0 / std::sqrt((double)D) : 0.0, nullptr, dtype, stream);
+}
+
+int swa_forward_host(const void* q, const void* k, const void* v, void* out, void* dq, void* dk, void* dv,
+                     void* dout, int64_t B, int64_t H, int64_t T, int64_t D, int64_t W, int64_t heads_per_group,
+                     int dtype, void* stream) {
+    const char* fn = "swa_forward_host";
+    const double scale = D >= 1 ? 1.0 / std::sqrt((double)D) : 0.0;
+    int64_t st[4][3];
+    if (int rc = swa_internal::check_forward(fn, dq, dk, dv, dout, B, H, T, D, W, scale, nullptr, dtype, st))
+        return rc;
+    if (B == 0 || H == 0 || T == 0) return success();
+    if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "%s: null host pointer", fn);
+    if (heads_per_group < 0) return fail(SWA_ERR_INVALID_ARG, "%s: heads_per_group < 0", fn);
+    const int64_t BH = B * H;
+    int64_t hpg = heads_per_group > 0 ? heads_per_group : (BH + 7) / 8;  // about 8 groups
+    if (hpg > BH) hpg = BH;
+    const int64_t n_groups = (BH + hpg - 1) / hpg;
+    const size_t head_bytes = (size_t)T * (size_t)D * (dtype == SWA_BF16 ? 2 : 4);
+    int dev;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    HostPipe* hp = &host_pipe(dev);
+    std::lock_guard<std::mutex> lk(hp->mu);
+    if (int rc = host_pipe_ready(*hp, (size_t)(2 * n_groups + 2))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t* ev = hp->ev.data();  // [0] start, [1] done, then (copied in, computed) per group
+    auto bytes_at = [&](const void* base, int64_t g0) {
+        return static_cast<const char*>(base) + (size_t)g0 * head_bytes;
+    };
+    // everything already on the caller's stream (earlier users of the staging buffers) first
+    if ((e = cudaEventRecord(ev[0], s)) != cudaSuccess || (e = cudaStreamWaitEvent(hp->in, ev[0], 0)) != cudaSuccess)
+        return cuda_fail(e, "swa_forward_host: ordering after the caller's stream");
+    for (int64_t g = 0; g < n_groups; ++g) {
+        const int64_t g0 = g * hpg, nh = (g0 + hpg <= BH ? hpg : BH - g0);
+        const size_t nb = (size_t)nh * head_bytes;
+        cudaEvent_t e_in = ev[2 + 2 * g], e_cmp = ev[3 + 2 * g];
+        // the (b, h) heads are independent problems: heads g0 .. g0+nh-1 of the contiguous
+        // [B,H,T,D] tensors are one [1, nh, T, D] problem
+        if ((e = cudaMemcpyAsync(const_cast<char*>(bytes_at(dq, g0)), bytes_at(q, g0), nb, cudaMemcpyHostToDevice, hp->in)) ||
+            (e = cudaMemcpyAsync(const_cast<char*>(bytes_at(dk, g0)), bytes_at(k, g0), nb, cudaMemcpyHostToDevice, hp->in)) ||
+            (e = cudaMemcpyAsync(const_cast<char*>(bytes_at(dv, g0)), bytes_at(v, g0), nb, cudaMemcpyHostToDevice, hp->in)) ||
+            (e = cudaEventRecord(e_in, hp->in)) || (e = cudaStreamWaitEvent(hp->cmp, e_in, 0)))
+            return cuda_fail(e, "swa_forward_host: host-to-device copies");
+        if (int rc = forward_impl(fn, bytes_at(dq, g0), bytes_at(dk, g0), bytes_at(dv, g0),
+                                  const_cast<char*>(bytes_at(dout, g0)), 1, nh, T, D, W, scale, nullptr, dtype,
+                                  hp->cmp))
+            return rc;
+        if ((e = cudaEventRecord(e_cmp, hp->cmp)) || (e = cudaStreamWaitEvent(hp->out, e_cmp, 0)) ||
+            (e = cudaMemcpyAsync(const_cast<char*>(bytes_at(out, g0)), bytes_at(dout, g0), nb, cudaMemcpyDeviceToHost,
+                                 hp->out)))
+            return cuda_fail(e, "swa_forward_host: device-to-host copy");
+    }
+    if ((e = cudaEventRecord(ev[1], hp->out)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ev[1], 0)) != cudaSuccess)
+        return cuda_fail(e, "swa_forward_host: ordering the caller's stream after the copies");
+    return success();
 }
 
 int swa_forward_ex(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t H,
@@ -873,7 +980,11 @@ extern "C" int swa_decode_noalloc(const void* q, const void* kring, const void* 
         if (int rc = noalloc_scratch(&base)) return rc;
         counters = static_cast<int*>(base);
         part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + counter_bytes);
-        // the array keeps the last call's contents: the ticket counters must start at zero
+        // The array keeps the last call's contents and the ticket counters must start at
+        // zero. Every decode kernel that runs to its end puts its counters back to zero, so
+        // after ordered calls they already are; the clear guards against a launch that
+        // never ran to its end (a kernel stopped by an error), at the cost of one memset
+        // node of B*H*4 bytes per call.
         cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)(B * H) * sizeof(int), s);
         if (e != cudaSuccess) return cuda_fail(e, "swa_decode_noalloc: clearing counters");
     }
