@@ -91,6 +91,56 @@ def test_tile_class_rejects_bad_args():
     assert swa.tile_class(100, 3, 128, 128, 1, 0) == -1
 
 
+def _pair_tiles(T, W, p):
+    """Visited 128 x 128 tiles of the pair of query tiles (2p, 2p+1), by enumeration."""
+    n_qt = (T + 127) // 128
+    return sum(1 for qt in (2 * p, 2 * p + 1) if qt < n_qt
+               for kt in range(n_qt) if swa.tile_class(T, W, 128, 128, qt, kt) > 0)
+
+
+@pytest.mark.parametrize("B,H,T,W", [(1, 32, 16384, 4096), (2, 16, 8192, 1), (2, 16, 8192, 1024),
+                                     (2, 16, 8192, 8192), (1, 8, 512, 128), (1, 3, 1000, 129),
+                                     (2, 3, 1300, 5000), (1, 2, 129, 64), (3, 1, 640, 300)])
+def test_work_items_cover_every_pair_once_heads_grouped(B, H, T, W):
+    """The prefill's work items are a permutation of all (b, h, pair); the equal-work
+    pairs come first, head after head; the rest follow with non-increasing work; and the
+    snake assignment over min(items, 148) CTAs gives every CTA about the mean work."""
+    n_qt = (T + 127) // 128
+    n_pairs = (n_qt + 1) // 2
+    n = B * H * n_pairs
+    items = [swa.work_item(u, B, H, T, W) for u in range(n)]
+    assert sorted(items) == sorted((b, h, p) for b in range(B) for h in range(H) for p in range(n_pairs))
+    assert swa.work_item(n, B, H, T, W) is None and swa.work_item(-1, B, H, T, W) is None
+    w = min(W, T)
+    full = [(b, h, p) for (b, h, p) in items if 256 * p >= w - 1 and 2 * p + 1 < n_qt]
+    nf = len(full)
+    assert items[:nf] == full, "the whole-window pairs come first"
+    heads = [b * H + h for (b, h, _) in full]
+    assert heads == sorted(heads), "head after head"
+    work = {p: _pair_tiles(T, W, p) for p in range(n_pairs)}
+    assert len({work[p] for (_, _, p) in full}) <= 1, "the first section is equal work"
+    rest = [work[p] for (_, _, p) in items[nf:]]
+    assert rest == sorted(rest, reverse=True), "the rest heaviest first"
+    G = min(n, 148)
+    per_cta = np.zeros(G)
+    for g in range(G):
+        r = 0
+        while True:
+            u = r * G + ((G - 1 - g) if r & 1 else g)
+            if u >= n:
+                break
+            per_cta[g] += work[items[u][2]]
+            r += 1
+    if n >= 4 * G:  # several items per CTA
+        assert per_cta.max() <= 1.08 * per_cta.mean()
+
+
+def test_work_item_rejects_bad_args():
+    assert swa.work_item(0, 0, 1, 10, 3) is None
+    assert swa.work_item(0, 1, 1, 0, 3) is None
+    assert swa.work_item(0, 1, 1, 10, 0) is None
+
+
 def test_valid_slots_match_ring_enumeration():
     for W in (1, 2, 3, 7, 64):
         for pos in list(range(0, 3 * W + 2)) + [W - 2, W - 1, W, 10**6 + 3]:

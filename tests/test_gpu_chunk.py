@@ -158,23 +158,3 @@ def test_stream_errors():
     assert a(p, p, rp + 8, rp, pp, 1, 1, 8, 64, 16, s) == 3
     assert a(p, p, rp, rp, pp, 0, 1, 8, 64, 16, s) == 0
     swa.device_status()
-
-
-def test_chunk_workload_full_size_sampled():
-    """The full chunked streaming workload (B64 H32 C128 D128 W4096, positions uniform
-    in [0, 100000)): every row of sampled streams against the oracle, and their rings
-    after the append bit for bit."""
-    wl = inputs.CHUNKED
-    q, k, v, kr, vr, pos = inputs.for_workload(wl)
-    dk, dv = kr.to(DEV), vr.to(DEV)
-    out = swa.chunk_forward(q.to(DEV), k.to(DEV), v.to(DEV), dk, dv, pos.to(DEV), wl.W)
-    swa.device_status()
-    for b in (0, 17, int(torch.argmin(pos)), 63):
-        for h in (0, 31):
-            sl = (slice(b, b + 1), slice(h, h + 1))
-            ref = oracle.chunk(f64(q[sl]), f64(k[sl]), f64(v[sl]), f64(kr[sl]), f64(vr[sl]),
-                               pos.numpy()[b:b + 1], wl.W)
-            assert max_err(out[sl], ref) <= TOL[BF], f"stream b={b} h={h} (pos {int(pos[b])})"
-            ek, ev = oracle.ring_append(f64(k[sl]), f64(v[sl]), f64(kr[sl]), f64(vr[sl]),
-                                        pos.numpy()[b:b + 1], wl.W)
-            assert np.array_equal(f64(dk[sl]), ek) and np.array_equal(f64(dv[sl]), ev)

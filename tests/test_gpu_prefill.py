@@ -9,7 +9,7 @@ import oracle
 import sliding_window_causal_b200 as swa
 from sliding_window_causal_b200 import _native, inputs
 from golden import read_moving_average
-from gpu_util import TOL, f64, max_err, oracle_rows, sample_rows
+from gpu_util import TOL, f64, max_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -172,34 +172,19 @@ def test_timeout_path_reports_and_recovers():
 
 
 # ---------------------------------------------------------------- full-size workloads
+# Every element of the full-size workloads is compared in test_gpu_fullsize.py; here the
+# properties that hold at any size, over every output of the Mistral-shaped workload.
 
-def sampled_parity(wl, heads, n_random=96):
+def test_mistral_shaped_properties():
+    wl = inputs.MISTRAL
     q, k, v = inputs.for_workload(wl)
     out = swa.forward(q.to(DEV), k.to(DEV), v.to(DEV), wl.W)
     swa.device_status()
-    rows = sample_rows(wl.T, wl.W, n_random=n_random, seed=wl.seed)
-    refs = oracle_rows(q, k, v, wl.W, heads, rows)
-    worst = 0.0
-    for (b, h), ref in refs.items():
-        got = out[b, h, torch.from_numpy(rows).to(DEV)]
-        worst = max(worst, max_err(got, ref))
-    assert worst <= TOL[wl.dtype], f"{wl.name}: max err {worst}"
-    # properties at any size, over every output: finite, and each output a convex
-    # combination of v rows, so no larger in magnitude than the largest |v|
+    # finite, and each output a convex combination of v rows, so no larger in magnitude
+    # than the largest |v|
     assert bool(torch.isfinite(out).all())
     vmax = v.abs().max().item()
     assert out.abs().max().item() <= vmax * (1 + 2 ** -8)
-    return worst
-
-
-def test_mistral_shaped_sampled():
-    wl = inputs.MISTRAL
-    sampled_parity(wl, [(0, 0), (0, 13), (0, 31)])
-
-
-@pytest.mark.parametrize("wl", inputs.SWEEP, ids=lambda w: w.name)
-def test_window_sweep_sampled(wl):
-    sampled_parity(wl, [(0, 0), (1, 15)], n_random=48)
 
 
 @pytest.mark.parametrize("D,W", [(128, 4096), (64, 700), (128, 200)])
@@ -208,16 +193,16 @@ def test_growing_scores_move_the_reference(D, W):
     row's running maximum up by far more than the lazy-rescale threshold, tile after
     tile; the output must still match.
 
-    Here a handful of keys dominate every row, so |out| is close to a single |v|. v is
-    drawn at half scale to keep |out| below about 1.5: at |out| >= 2 the bf16 output
-    spacing alone (0.0156) leaves half the 1e-2 budget to the bf16 weights P, which is
-    a property of bf16 outputs and bf16 P, not of the rescale path tested here."""
+    A handful of keys dominate every row, so |out| comes close to a single |v| and can
+    pass 2, where the bf16 output spacing alone costs up to 0.0078 of the 1e-2 budget.
+    These are the rows the kernel recomputes in fp32 (a key of a single-bf16 tile holds
+    more than 1/16 of the row's weight); v is drawn at full scale, N(0, 1)."""
     T = 1500
     gen = torch.Generator().manual_seed(71)
     q = torch.ones(1, 2, T, D)
     k = (torch.arange(T, dtype=torch.float32) * 0.05)[None, None, :, None].expand(1, 2, T, D).clone()
     k += 0.01 * torch.randn(1, 2, T, D, generator=gen)
-    v = 0.5 * torch.randn(1, 2, T, D, generator=gen)
+    v = torch.randn(1, 2, T, D, generator=gen)
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
     out = run(q, k, v, W)
     ref = oracle.forward(f64(q), f64(k), f64(v), W)
