@@ -12,8 +12,9 @@
 //   warp 0, lane 0   TMA producer: the Q tile, then K and V of every visited key tile
 //                    through an NSTAGE ring: first the ring's slot tiles (128 slots each),
 //                    then the chunk's key tiles.
-//   warp 1           allocates TMEM; lane 0 issues the tcgen05 MMAs. S is double
-//                    buffered, S_j = Q K_j^T -> TMEM columns [128 + 128(j&1), +128), and the
+//   warp 1           allocates TMEM; the warp runs the MMA loop and an elected lane issues
+//                    the tcgen05 MMAs. S is double buffered,
+//                    S_j = Q K_j^T -> TMEM columns [128 + 128(j&1), +128), and the
 //                    order S_0, S_1, PV_0, S_2, PV_1, ... computes S_{j+1} while the softmax
 //                    works on S_j, so the softmax never waits for its own P.V product.
 //                    O += P_j V_j accumulates in TMEM columns [0, D).
@@ -226,8 +227,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {
             // ---------------------------------------------------------------- MMA issuer
+            // (the whole warp runs this loop; its waits are warp-uniform, one lane issues)
             const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
             const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
             const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
@@ -239,50 +241,50 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             int n = 0;
             for (int t = 0; t < it.n_st; ++t) n += chunk_ring_class(it, W, t) != 0;
             n += it.kl - it.kf + 1;
-            bool ok = ptx::mbar_wait(q_full, 0, wait_limit_ns, abort_flag);
+            bool ok = pp_wait_warp(q_full, 0, wait_limit_ns, abort_flag);
             auto issue_s = [&](int j) {
                 const uint32_t L = 2u * j, st = L % NS;
-                ok = ptx::mbar_wait(ring_full + st, (L / NS) & 1, wait_limit_ns, abort_flag);
+                ok = pp_wait_warp(ring_full + st, (L / NS) & 1, wait_limit_ns, abort_flag);
                 if (!ok) return;
                 ptx::tc_fence_after();
                 const uint32_t k_lo = (ring_lo + st * kStageLo) | lo_k;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + Cfg::colS(j & 1), desc_hi | (q_lo + off), desc_hi | (k_lo + off), idesc_s,
+                    ptx::mma_ss_one(tmem + Cfg::colS(j & 1), desc_hi | (q_lo + off), desc_hi | (k_lo + off), idesc_s,
                                 kk > 0 ? 1u : 0u);
                 }
-                ptx::tc_commit(s_full + (j & 1));
-                ptx::tc_commit(ring_empty + st);  // K_j read
+                ptx::tc_commit_one(s_full + (j & 1));
+                ptx::tc_commit_one(ring_empty + st);  // K_j read
             };
             auto issue_pv = [&](int j) {
-                ok = ptx::mbar_wait(p_full + (j & 1), (j >> 1) & 1, wait_limit_ns, abort_flag);
+                ok = pp_wait_warp(p_full + (j & 1), (j >> 1) & 1, wait_limit_ns, abort_flag);
                 const uint32_t L = 2u * j + 1, st = L % NS;
-                if (ok) ok = ptx::mbar_wait(ring_full + st, (L / NS) & 1, wait_limit_ns, abort_flag);
+                if (ok) ok = pp_wait_warp(ring_full + st, (L / NS) & 1, wait_limit_ns, abort_flag);
                 if (!ok) return;
                 ptx::tc_fence_after();
                 const uint32_t v_lo = (ring_lo + st * kStageLo) | lo_v;
                 const uint32_t scol = tmem + Cfg::colS(j & 1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_ts(tmem + Cfg::kColO, scol + pp_pcol(kk), desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
+                    ptx::mma_ts_one(tmem + Cfg::kColO, scol + pp_pcol(kk), desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
                                 (j > 0 || kk > 0) ? 1u : 0u);
                 if (it.precise) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tmem + Cfg::kColO, scol + pp_pcol(kk) + 16, desc_hi | (v_lo + kk * (2048 >> 4)),
+                        ptx::mma_ts_one(tmem + Cfg::kColO, scol + pp_pcol(kk) + 16, desc_hi | (v_lo + kk * (2048 >> 4)),
                                     idesc_o, 1u);
                 }
-                ptx::tc_commit(pv_done);
-                ptx::tc_commit(ring_empty + st);  // V_j read
-                if (j == n - 1) ptx::tc_commit(o_final);
+                ptx::tc_commit_one(pv_done);
+                ptx::tc_commit_one(ring_empty + st);  // V_j read
+                if (j == n - 1) ptx::tc_commit_one(o_final);
             };
             if (ok) issue_s(0);
             for (int j = 0; j < n && ok; ++j) {
                 if (j + 1 < n) issue_s(j + 1);
                 if (ok) issue_pv(j);
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 atomicCAS(status, 0, 5);
                 *abort_flag = 1;
             }
@@ -402,8 +404,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);
             }
         }
-        if (warp == 1 && lane == 0) {
-            ptx::tc_commit(drain);  // completes when every MMA issued so far is done
+        if (warp == 1) {
+            ptx::tc_commit_one(drain);  // completes when every MMA issued so far is done
             ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
         }
         __syncthreads();

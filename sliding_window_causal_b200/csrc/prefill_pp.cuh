@@ -20,9 +20,12 @@
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0, lane 0     TMA producer: Q_A, Q_B per item, then K_kt and V_kt through one
 //                      NSTAGE-deep ring of 128-row tiles.
-//   warp 1             allocates the 512 TMEM columns; the warp runs the MMA loop and an
-//                      elected lane issues every tcgen05 MMA in the order PV_A(kt-1),
-//                      S_A(kt), PV_B(kt-1), S_B(kt), so that the tensor
+//   warp 1 (and 3)     warp 1 allocates the 512 TMEM columns. With one issuer (TWO = false)
+//                      the whole of warp 1 runs the MMA loop and an elected lane issues every
+//                      tcgen05 MMA in the order PV_A(kt-1), S_A(kt), PV_B(kt-1), S_B(kt); with
+//                      two (TWO = true, for short bands), warp 1 issues tile A's products and
+//                      warp 3 tile B's, each in the order S_x(kt), PV_x(kt), S_x(kt+1), ...
+//                      Either way the tensor
 //                      core works on one tile's products while the other tile's softmax runs:
 //                        S_X = Q_X K^T   -> TMEM columns [128X, 128X+128)   (fp32)
 //                        O_X += P_X V    -> TMEM columns [256+128X, +D)     (fp32)
@@ -69,9 +72,11 @@ constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow
 // use up the error budget left by the output's own bf16 rounding.
 constexpr int kPPPreciseWindow = 32;
 constexpr uint64_t kPPDrainLimitNs = 200000000ull;
+// Bands of at most this many keys use two MMA issuers (one per query tile), longer ones one.
+constexpr int kPPTwoIssuerWindow = 1024;
 // P of a tile is handed to the MMA issuer in this many parts (1, 2 or 4), so that the
 // first keys' P.V products run while the softmax still works on the last keys.
-constexpr int kPPParts = 4;
+constexpr int kPPParts = 2;
 static_assert(kPPParts == 1 || kPPParts == 2 || kPPParts == 4, "parts of a tile's P");
 // A row whose largest weight from a single-bf16-P tile ends up above kPPSharpShare of the
 // row's total weight, and one of whose outputs reaches kPPSharpOut in magnitude, is
@@ -102,9 +107,9 @@ struct PPCfg {
     static constexpr int kQOff = 0;                    // Q_A, Q_B
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-    // q_full[2], q_empty[2], ring_full[S], ring_empty[S], s_full[2], p_full[2][4],
-    // o_final[2], o_free[2], drain
-    static constexpr int kNumBars = 4 + 2 * kStages + 15;
+    // q_full[2], q_empty[2], ring_full[S], ring_empty[2][S], s_full[2], p_full[2][4],
+    // o_final[2], o_free[2], drain[2]
+    static constexpr int kNumBars = 4 + 3 * kStages + 16;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, 4 queue counters
     static constexpr int kFixOff = (kMiscOff + 24 + 15) & ~15;  // queue of sharp rows: kPPFixSlots x 16 B
     static constexpr int kSmemBytes = kFixOff + kPPFixSlots * 16 + 1024;  // + alignment slack
@@ -426,7 +431,7 @@ __device__ __forceinline__ bool pp_push_sharp(uint32_t* fix_head, const uint32_t
 
 // LSE: also write the natural log-sum-exp of each row (a separate instantiation, so that
 // the plain prefill keeps its register allocation).
-template <int D, bool LSE = false>
+template <int D, bool LSE = false, bool TWO = false>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
@@ -442,12 +447,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     uint64_t* q_full = bars;            // [2]
     uint64_t* q_empty = bars + 2;       // [2]
     uint64_t* ring_full = bars + 4;     // [NS]
-    uint64_t* ring_empty = ring_full + NS;
-    uint64_t* s_full = ring_empty + NS;  // [2]
+    uint64_t* ring_empty = ring_full + NS;  // [2][NS]: tile x's issuer is done with the stage
+    uint64_t* s_full = ring_empty + 2 * NS;  // [2]
     uint64_t* p_full = s_full + 2;       // [2][4]: P of tile x, part s, is in TMEM
     uint64_t* o_final = p_full + 8;      // [2]
     uint64_t* o_free = o_final + 2;      // [2]
-    uint64_t* drain = o_free + 2;
+    uint64_t* drain = o_free + 2;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
     // queue of sharp rows: fix_head counts the rows pushed, fix_tail the rows the worker has
@@ -475,8 +480,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(ring_full + s, 1);
             ptx::mbar_init(ring_empty + s, 1);
+            ptx::mbar_init(ring_empty + NS + s, 1);
         }
         ptx::mbar_init(drain, 1);
+        ptx::mbar_init(drain + 1, 1);
         *abort_flag = 0;
         *fix_head = 0;
         *fix_done = 0;
@@ -527,7 +534,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     for (int kv = 0; kv < 2; ++kv) {
                         const uint32_t st = loads % NS;
                         if (loads >= (uint32_t)NS)
-                            ok = ptx::mbar_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag);
+                            ok = ptx::mbar_wait(ring_empty + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag) &&
+                                 (!TWO ||
+                                  ptx::mbar_wait(ring_empty + NS + st, ((loads / NS) - 1) & 1, wait_limit_ns, abort_flag));
                         if (!ok) break;
                         uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
                         ptx::mbar_arrive_expect_tx(ring_full + st, C::kTileBytes);
@@ -543,9 +552,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 *abort_flag = 1;
             }
         }
-    } else if (warp == 1) {
+    } else if (!TWO && warp == 1) {
         {
-            // ------------------------------------------------------------ MMA issuer
+            // ------------------------------------------------------------ MMA issuer (one warp)
             // (the whole warp runs this loop; its waits are warp-uniform, one lane issues)
             // Descriptors: the high word (SBO = 1024, sm_100 version, 128-byte swizzle) is
             // the same for every operand; the low word is start >> 4 plus the leading byte
@@ -641,6 +650,119 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 L = Lbase + 2u * (uint32_t)(it.k1 - it.k0 + 1);
                 ++ni[0];
                 if (it.hasB) ++ni[1];
+            }
+            if (!ok && lane == 0) {
+                atomicCAS(status, 0, 5);
+                *abort_flag = 1;
+            }
+        }
+    } else if (TWO && (warp == 1 || warp == 3)) {
+        {
+            // ------------------------------------------------------------ MMA issuers (two warps)
+            // Warp 1 issues tile A's products, warp 3 tile B's, each as a whole warp
+            // (warp-uniform waits, one elected lane issues): S_x(f), PV_x(f), S_x(f+1), ...
+            // Two issuers keep one tile's wait for its P from holding up the other tile's
+            // products. Each issuer releases every ring stage of the item, used or not, on its
+            // own ring_empty barrier (after the products that read it, or once the stage is
+            // filled if it does not use it), so the producer waits for both.
+            // Descriptors: the high word (SBO = 1024, sm_100 version, 128-byte swizzle) is
+            // the same for every operand; the low word is start >> 4 plus the leading byte
+            // offset field, so each MMA needs one add (shared memory is far below 256 KiB, so
+            // start >> 4 + offset never carries out of its 14-bit field).
+            const int x = warp == 1 ? 0 : 1;
+            const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
+            const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
+            const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
+            const uint32_t lo_k = (uint32_t)umma::smem_desc(0, 16, 1024);              // K-major LBO field
+            const uint32_t lo_v = (uint32_t)umma::smem_desc(0, C::kBoxBytes, 1024);   // MN-major LBO field
+            const uint32_t q_lo = (ptx::smem_u32(smem + C::kQOff + x * C::kTileBytes) >> 4) | lo_k;
+            const uint32_t ring_lo = ptx::smem_u32(smem + C::kRingOff) >> 4;
+            constexpr uint32_t kStageLo = C::kTileBytes >> 4;
+            uint64_t* my_empty = ring_empty + x * NS;
+            const auto release = [&](uint32_t st, bool used) {
+                if (used) ptx::tc_commit_one(my_empty + st);  // once the products that read it are done
+                else if (lane == 0) ptx::mbar_arrive(my_empty + st);
+            };
+            uint32_t L = 0;   // K/V tiles consumed so far (same count as the producer)
+            int ni = 0;       // items of this tile seen
+            uint32_t ns = 0;  // S tiles issued
+            bool ok = true;
+            for (int r = 0; ok; ++r) {
+                const int u = pp_item(r, g, G, n_items);
+                if (u < 0) break;
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
+                const bool mine = x == 0 || it.hasB;
+                const int f = it.f[x], l = it.l[x];
+                const bool prec = pp_precise(it.qt[x], W);
+                if (mine) ok = pp_wait_warp(q_full + x, ni & 1, wait_limit_ns, abort_flag);
+                if (!ok) break;
+                int pend = -1;
+                bool first_pv = true;
+                const uint32_t Lbase = L;
+                for (int kt = it.k0; kt <= it.k1 + 1 && ok; ++kt) {
+                    const uint32_t j = (uint32_t)(kt - it.k0);
+                    const uint32_t Lk = Lbase + 2 * j, Lv = Lk - 1;
+                    if (kt > it.k0) {
+                        // PV_x(kt-1) (before S_x(kt), which overwrites P_x(kt-1)); V(kt-1) released
+                        const uint32_t stv = Lv % NS;
+                        ok = pp_wait_warp(ring_full + stv, (Lv / NS) & 1, wait_limit_ns, abort_flag);
+                        if (ok && pend >= 0) {
+                            // part by part as the softmax hands P_x(kt-1) over; O_x must be
+                            // free if it starts the item
+                            if (first_pv && ni > 0)
+                                ok = pp_wait_warp(o_free + x, (ni - 1) & 1, wait_limit_ns, abort_flag);
+                            const uint32_t v_lo = (ring_lo + stv * kStageLo) | lo_v;
+#pragma unroll
+                            for (int part = 0; part < kPPParts && ok; ++part) {
+                                ok = pp_wait_warp(p_full + 4 * x + part, (ns - 1) & 1, wait_limit_ns, abort_flag);
+                                if (!ok) break;
+                                ptx::tc_fence_after();
+                                constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
+#pragma unroll
+                                for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                    ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
+                                                    desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
+                                                    (!first_pv || kk > 0) ? 1u : 0u);
+                                if (prec) {
+#pragma unroll
+                                    for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                        ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                        desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u);
+                                }
+                            }
+                            if (!ok) break;
+                            first_pv = false;
+                            if (pend == l) ptx::tc_commit_one(o_final + x);
+                        }
+                        if (!ok) break;
+                        release(stv, pend >= 0);
+                        pend = -1;
+                    }
+                    if (kt <= it.k1) {
+                        // S_x(kt) = Q_x K(kt)^T; K(kt) released
+                        const uint32_t stk = Lk % NS;
+                        ok = pp_wait_warp(ring_full + stk, (Lk / NS) & 1, wait_limit_ns, abort_flag);
+                        if (!ok) break;
+                        const bool use = mine && kt >= f && kt <= l;
+                        if (use) {
+                            ptx::tc_fence_after();
+                            const uint32_t k_lo = (ring_lo + stk * kStageLo) | lo_k;
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                                ptx::mma_ss_one(tmem + C::colS(x), desc_hi | (q_lo + off), desc_hi | (k_lo + off),
+                                                idesc_s, kk > 0 ? 1u : 0u);
+                            }
+                            ptx::tc_commit_one(s_full + x);
+                            ++ns;
+                            if (kt == l) ptx::tc_commit_one(q_empty + x);
+                            pend = kt;
+                        }
+                        release(stk, use);
+                    }
+                }
+                L = Lbase + 2u * (uint32_t)(it.k1 - it.k0 + 1);
+                if (mine) ++ni;
             }
             if (!ok && lane == 0) {
                 atomicCAS(status, 0, 5);
@@ -827,9 +949,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);
             }
         }
-        if (warp == 1) {
-            ptx::tc_commit_one(drain);  // completes when every MMA issued so far is done
-            ptx::mbar_wait(drain, 0, kPPDrainLimitNs, nullptr);
+        if (warp == 1 || (TWO && warp == 3)) {
+            const int x = warp == 1 ? 0 : 1;
+            ptx::tc_commit_one(drain + x);  // completes when every MMA this warp issued is done
+            ptx::mbar_wait(drain + x, 0, kPPDrainLimitNs, nullptr);
         }
         __syncthreads();
     }

@@ -82,6 +82,19 @@ struct DeviceState {
 };
 std::map<int, DeviceState> g_dev;
 
+// The eight tensor-core prefill kernels (D 64/128, with and without the log-sum-exp, one or
+// two MMA issuers): set the shared-memory size, and check that each was compiled with the
+// kPPLaunchRegs registers per thread that its register split assumes.
+template <int D, bool LSE, bool TWO>
+cudaError_t set_pp_attrs(bool* regs_ok) {
+    cudaError_t e = cudaFuncSetAttribute(swa::prefill_pp_kernel<D, LSE, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         swa::PPCfg<D>::kSmemBytes);
+    cudaFuncAttributes a;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, swa::prefill_pp_kernel<D, LSE, TWO>);
+    if (e == cudaSuccess && a.numRegs != swa::kPPLaunchRegs) *regs_ok = false;
+    return e;
+}
+
 template <int D>
 cudaError_t set_bwd_tc_attrs() {
     cudaError_t e = cudaFuncSetAttribute(swa::bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -116,22 +129,16 @@ int device_state(DeviceState** out) {
     }
     if (!st.attrs_set) {
         e = cudaSuccess;
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<128>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::PPCfg<128>::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::PPCfg<64>::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<128, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::PPCfg<128>::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(swa::prefill_pp_kernel<64, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::PPCfg<64>::kSmemBytes);
+        bool regs_ok = true;  // the register split inside the kernels assumes this launch allocation
+        if (e == cudaSuccess) e = set_pp_attrs<128, false, false>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<128, true, false>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<128, false, true>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<128, true, true>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<64, false, false>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<64, true, false>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<64, false, true>(&regs_ok);
+        if (e == cudaSuccess) e = set_pp_attrs<64, true, true>(&regs_ok);
+        st.pp_regs_ok = e == cudaSuccess && regs_ok;
         if (e == cudaSuccess) e = set_bwd_tc_attrs<64>();
         if (e == cudaSuccess) e = set_bwd_tc_attrs<128>();
         if (e == cudaSuccess) e = set_bwd_attrs<float>();
@@ -144,17 +151,6 @@ int device_state(DeviceState** out) {
                                      swa::ChunkCfg<64>::kSmemBytes);
         if (e == cudaSuccess)
             e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess) {
-            // The register split inside the kernel assumes this launch allocation.
-            cudaFuncAttributes a128, a64, l128, l64;
-            e = cudaFuncGetAttributes(&a128, swa::prefill_pp_kernel<128>);
-            if (e == cudaSuccess) e = cudaFuncGetAttributes(&a64, swa::prefill_pp_kernel<64>);
-            if (e == cudaSuccess) e = cudaFuncGetAttributes(&l128, swa::prefill_pp_kernel<128, true>);
-            if (e == cudaSuccess) e = cudaFuncGetAttributes(&l64, swa::prefill_pp_kernel<64, true>);
-            st.pp_regs_ok = e == cudaSuccess && a128.numRegs == swa::kPPLaunchRegs &&
-                            a64.numRegs == swa::kPPLaunchRegs && l128.numRegs == swa::kPPLaunchRegs &&
-                            l64.numRegs == swa::kPPLaunchRegs;
-        }
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(swa::prefill_simt_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -395,22 +391,23 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
             raw.sk[x] = st[1][x];
             raw.sv[x] = st[2][x];
         }
-        if (D == 128 && lse)
-            swa::prefill_pp_kernel<128, true><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status, raw);
-        else if (D == 128)
-            swa::prefill_pp_kernel<128><<<G, swa::kPPThreads, swa::PPCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status, raw);
-        else if (lse)
-            swa::prefill_pp_kernel<64, true><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status, raw);
-        else
-            swa::prefill_pp_kernel<64><<<G, swa::kPPThreads, swa::PPCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], nullptr, (int)BH, (int)H, (int)T, Wi, n_qt,
-                scale_log2, wait_limit(), ds->status, raw);
+        // Bands of at most kPPTwoIssuerWindow keys are short: an item's pipeline fills and
+        // drains every few tiles, and one MMA issuer per query tile keeps either tile from
+        // waiting on the other's P. Longer bands keep the single issuer, whose ping-pong order
+        // completes each tile's scores sooner.
+        const bool two = Wi <= swa::kPPTwoIssuerWindow;
+        auto launch = [&](auto kern, int smem) {
+            kern<<<G, swa::kPPThreads, smem, s>>>(mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H,
+                                                 (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status, raw);
+        };
+        constexpr int S128 = swa::PPCfg<128>::kSmemBytes, S64 = swa::PPCfg<64>::kSmemBytes;
+        if (D == 128) {
+            if (lse) two ? launch(swa::prefill_pp_kernel<128, true, true>, S128) : launch(swa::prefill_pp_kernel<128, true, false>, S128);
+            else two ? launch(swa::prefill_pp_kernel<128, false, true>, S128) : launch(swa::prefill_pp_kernel<128, false, false>, S128);
+        } else {
+            if (lse) two ? launch(swa::prefill_pp_kernel<64, true, true>, S64) : launch(swa::prefill_pp_kernel<64, true, false>, S64);
+            else two ? launch(swa::prefill_pp_kernel<64, false, true>, S64) : launch(swa::prefill_pp_kernel<64, false, false>, S64);
+        }
     } else {
         const int64_t nrows = B * H * T;
         const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;

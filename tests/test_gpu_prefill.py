@@ -46,6 +46,9 @@ BF16_SHAPES = [
     (1, 2, 1000, 128, 129), (1, 2, 777, 128, 300), (1, 1, 1000, 128, 1000),
     (1, 1, 1000, 128, 5000), (1, 2, 129, 64, 2), (1, 1, 1, 128, 1), (1, 1, 5, 64, 3),
     (2, 3, 400, 64, 256), (1, 1, 2000, 128, 640), (1, 2, 1280, 64, 1),
+    # either side of the band length (1024 keys) where the kernel moves from two MMA
+    # issuers to one
+    (1, 2, 3000, 128, 1024), (1, 2, 3000, 128, 1025), (1, 2, 2000, 64, 1500),
 ]
 
 
