@@ -53,7 +53,7 @@ struct BwdTcCfg {
     static constexpr int kFixOff = 0;                 // two resident tiles
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kStatStages = 2;
-    static constexpr int kStatBytes = 2 * 128 * 4;    // lse2[128], delta[128]
+    static constexpr int kStatBytes = 2 * 128 * 4;    // nlse2[128], delta[128]
     static constexpr int kStatOff = kRingOff + kStages * kTileBytes;
     static constexpr int kBarOff = kStatOff + kStatStages * kStatBytes;
     // fix_full, ring_full[S], ring_empty[S], stat_full[2], stat_empty[2], s_full, p_full,
@@ -65,10 +65,11 @@ struct BwdTcCfg {
     static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 384;
 };
 
-// delta_i = sum_d dout_i[d] out_i[d] (fp32) and lse2_i = lse_i * log2(e), one warp per row.
+// delta_i = sum_d dout_i[d] out_i[d] (fp32) and nlse2_i = -lse_i * log2(e), one warp per row
+// (negated, so that the exponent s*c2 - lse*log2(e) is one fused multiply-add, s*c2 + nlse2).
 __global__ void __launch_bounds__(256)
     bwd_stats_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
-                     const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
+                     const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ delta,
                      int64_t BH, int T, int Tpad, int D) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(256)
     const int i = (int)(r - bh * Tpad);
     if (i >= T) {
         if (lane == 0) {
-            lse2[r] = INFINITY;
+            nlse2[r] = -INFINITY;  // padding rows: P = 0
             delta[r] = 0.f;
         }
         return;
@@ -90,34 +91,51 @@ __global__ void __launch_bounds__(256)
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) {
         delta[r] = acc;
-        lse2[r] = lse[bh * T + i] * 1.4426950408889634f;
+        nlse2[r] = lse[bh * T + i] * -1.4426950408889634f;
     }
 }
 
 // One chunk of 32 columns of one TMEM row, already in registers: scores s (fp32, raw q.k)
-// and dp, to bf16 P and dS = P (dp - delta), with P = exp2(s*c2 - lse2) where the column
-// is valid, else 0. Column t's lse2 and delta come from lse2_of(t), delta_of(t). On EDGE
-// tiles only columns cmin..cmax are valid (band membership of one row is an interval of
-// columns); other tiles are valid throughout. dS goes to columns dpcol .. dpcol+15 and,
-// when STORE_P, P to dpcol+16 .. dpcol+31 (both over dp values already read), leaving the
-// S columns free for the next tile's scores.
-template <bool STORE_P, bool EDGE, typename Lse, typename Delta>
+// and dp, to bf16 P and dS = P (dp - delta), with P = exp2(s*c2 + nlse2) where the column
+// is valid, else 0 (nlse2 = -lse in log2 units). COLSTATS: each column has its own nlse2
+// and delta (32 values each at col_nlse, col_delta in shared memory, 16-byte aligned);
+// else the row's row_nlse, row_delta apply to every column. On EDGE tiles only columns
+// cmin..cmax are valid (band membership of one row is an interval of columns); other tiles
+// are valid throughout. dS goes to columns dpcol .. dpcol+15 and, when STORE_P, P to
+// dpcol+16 .. dpcol+31 (both over dp values already read), leaving the S columns free for
+// the next tile's scores. Pairs of columns go through the packed f32x2 arithmetic.
+template <bool STORE_P, bool EDGE, bool COLSTATS>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], uint32_t dpcol,
-                                          float c2, Lse lse2_of, Delta delta_of, int cmin, int cmax) {
+                                          float c2, const float* col_nlse, const float* col_delta,
+                                          float row_nlse, float row_delta, int cmin, int cmax) {
     uint32_t ph[16], dh[16];
+    const ptx::f32x2 cc = {c2, c2};
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-        float p[2], ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int col = 2 * t + e;
-            float pe = ptx::ex2(fmaf(__uint_as_float(s[col]), c2, -lse2_of(col)));
-            if (EDGE && !(col >= cmin && col <= cmax)) pe = 0.f;
-            p[e] = pe;
-            ds[e] = pe * (__uint_as_float(dp[col]) - delta_of(col));
+    for (int t2 = 0; t2 < 16; t2 += 2) {
+        float4 nl4, dl4;
+        if (COLSTATS) {
+            nl4 = *reinterpret_cast<const float4*>(col_nlse + 2 * t2);
+            dl4 = *reinterpret_cast<const float4*>(col_delta + 2 * t2);
+        } else {
+            nl4 = make_float4(row_nlse, row_nlse, row_nlse, row_nlse);
+            dl4 = make_float4(row_delta, row_delta, row_delta, row_delta);
         }
-        ph[t] = ptx::pack_bf16x2(p[0], p[1]);
-        dh[t] = ptx::pack_bf16x2(ds[0], ds[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int t = t2 + u;
+            const ptx::f32x2 nl = u ? ptx::f32x2{nl4.z, nl4.w} : ptx::f32x2{nl4.x, nl4.y};
+            const ptx::f32x2 dl = u ? ptx::f32x2{dl4.z, dl4.w} : ptx::f32x2{dl4.x, dl4.y};
+            const ptx::f32x2 z = ptx::fma2({__uint_as_float(s[2 * t]), __uint_as_float(s[2 * t + 1])}, cc, nl);
+            ptx::f32x2 p = {ptx::ex2(z.x), ptx::ex2(z.y)};
+            if (EDGE) {
+                if (!(2 * t >= cmin && 2 * t <= cmax)) p.x = 0.f;
+                if (!(2 * t + 1 >= cmin && 2 * t + 1 <= cmax)) p.y = 0.f;
+            }
+            const ptx::f32x2 ds =
+                ptx::mul2(p, ptx::sub2({__uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1])}, dl));
+            ph[t] = ptx::pack_bf16x2(p.x, p.y);
+            dh[t] = ptx::pack_bf16x2(ds.x, ds.y);
+        }
     }
     ptx::tmem_st16(dpcol, dh);
     if (STORE_P) ptx::tmem_st16(dpcol + 16, ph);
@@ -149,12 +167,12 @@ __device__ __forceinline__ void bwd_store_row(uint32_t col, float a, __nv_bfloat
 
 // KV = true: bwd_kv_kernel (resident K, V; streamed Q, dO; dK, dV out).
 // KV = false: bwd_q_kernel (resident Q, dO; streamed K, V; dQ out).
-// Maps are 4-D {D, T, H, B} of contiguous [B,H,T,D] tensors. lse2/delta: [B*H, Tpad].
+// Maps are 4-D {D, T, H, B} of contiguous [B,H,T,D] tensors. nlse2/delta: [B*H, Tpad].
 template <int D, bool KV>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const float* __restrict__ lse2, const float* __restrict__ delta, __nv_bfloat16* __restrict__ g1,
+                  const float* __restrict__ nlse2, const float* __restrict__ delta, __nv_bfloat16* __restrict__ g1,
                   __nv_bfloat16* __restrict__ g2, int H, int T, int Tpad, int W, int n_t, float c, float c2,
                   uint64_t wait_limit_ns, int* status) {
     using Cf = BwdTcCfg<D>;
@@ -257,7 +275,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     ++loads;
                 }
                 if (KV && ok) {
-                    // the query tile's lse2 and delta (512 bytes each, contiguous in [B*H, Tpad])
+                    // the query tile's nlse2 and delta (512 bytes each, contiguous in [B*H, Tpad])
                     const uint32_t ss = stat_loads % 2;
                     if (stat_loads >= 2)
                         ok = ptx::mbar_wait(stat_empty + ss, ((stat_loads / 2) - 1) & 1, wait_limit_ns, abort_flag);
@@ -265,7 +283,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     uint8_t* dst = smem + Cf::kStatOff + ss * Cf::kStatBytes;
                     ptx::mbar_arrive_expect_tx(stat_full + ss, Cf::kStatBytes);
                     const int64_t off = (int64_t)bh * Tpad + 128 * yt;
-                    ptx::bulk_load(dst, lse2 + off, 512, stat_full + ss);
+                    ptx::bulk_load(dst, nlse2 + off, 512, stat_full + ss);
                     ptx::bulk_load(dst + 512, delta + off, 512, stat_full + ss);
                     ++stat_loads;
                 }
@@ -388,9 +406,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         const int r = quarter * 32 + lane;  // the TMEM lane = this thread's resident row
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
         const int xr = 128 * xt + r;         // key index (KV) or query index (Q)
-        float my_lse2 = 0.f, my_delta = 0.f;
+        float my_nlse2 = 0.f, my_delta = 0.f;
         if (!KV) {
-            my_lse2 = lse2[(int64_t)bh * Tpad + xr];  // +inf on padding rows: P = 0
+            my_nlse2 = nlse2[(int64_t)bh * Tpad + xr];  // -inf on padding rows: P = 0
             my_delta = delta[(int64_t)bh * Tpad + xr];
         }
         bool ok = true;
@@ -434,16 +452,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 ptx::reg_fence(dpv);
                 const int cmin = clo - 32 * cc, cmax = chi - 32 * cc;
                 if (KV) {
-                    const float* sl = sts + 32 * cc;
-                    auto lse_of = [&](int t) { return sl[t]; };
-                    auto delta_of = [&](int t) { return sl[128 + t]; };
-                    if (edge) bwd_chunk<true, true>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
-                    else bwd_chunk<true, false>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
+                    const float* sl = sts + 32 * cc;  // the columns' nlse2, then (at +128) their delta
+                    if (edge) bwd_chunk<true, true, true>(sv[x], dpv, dc, c2, sl, sl + 128, 0.f, 0.f, cmin, cmax);
+                    else bwd_chunk<true, false, true>(sv[x], dpv, dc, c2, sl, sl + 128, 0.f, 0.f, cmin, cmax);
                 } else {
-                    auto lse_of = [&](int) { return my_lse2; };
-                    auto delta_of = [&](int) { return my_delta; };
-                    if (edge) bwd_chunk<false, true>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
-                    else bwd_chunk<false, false>(sv[x], dpv, dc, c2, lse_of, delta_of, cmin, cmax);
+                    if (edge) bwd_chunk<false, true, false>(sv[x], dpv, dc, c2, nullptr, nullptr, my_nlse2, my_delta, cmin, cmax);
+                    else bwd_chunk<false, false, false>(sv[x], dpv, dc, c2, nullptr, nullptr, my_nlse2, my_delta, cmin, cmax);
                 }
             }
             ptx::tmem_st_wait();

@@ -791,11 +791,11 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
             (rc = make_map(&mv, v, B, H, T, D, cst)) || (rc = make_map(&mdo, dout, B, H, T, D, cst)))
             return rc;
         cudaStream_t s = static_cast<cudaStream_t>(stream);
-        float* lse2 = static_cast<float*>(workspace);
-        float* delta = lse2 + BH * Tpad;
+        float* nlse2 = static_cast<float*>(workspace);
+        float* delta = nlse2 + BH * Tpad;
         const int Wi = (int)(W < T ? W : T);
         swa::bwd_stats_kernel<<<(unsigned)((BH * Tpad + 7) / 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), lse, lse2, delta, BH,
+            static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), lse, nlse2, delta, BH,
             (int)T, (int)Tpad, (int)D);
         const float c = (float)scale, c2 = (float)(1.4426950408889634 * scale);
         const unsigned grid = (unsigned)(BH * n_t);
@@ -804,17 +804,17 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
         auto* gv = static_cast<__nv_bfloat16*>(dv);
         if (D == 128) {
             swa::bwd_tc_kernel<128, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, lse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
             swa::bwd_tc_kernel<128, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, lse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
         } else {
             swa::bwd_tc_kernel<64, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, lse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
             swa::bwd_tc_kernel<64, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, lse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
         }
         cudaError_t e = cudaGetLastError();
