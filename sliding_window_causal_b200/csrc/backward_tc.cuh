@@ -16,7 +16,10 @@
 //                     dS^T over the dP^T columns; then dV += P^T dO and dK += dS^T Q
 //                     accumulate in TMEM (TS form: A from TMEM, B from shared memory). The
 //                     next tile's S^T is computed while the element-wise warps work: they
-//                     read their scores into registers first and release the S columns.
+//                     read their scores into registers first and release the S columns. They
+//                     then take the tile's columns in two halves of 64; the gradient products
+//                     of a half, and the next tile's dP^T for that half, run on the tensor
+//                     cores while the warps work on the other half.
 //   bwd_tc_kernel<D, false>: one CTA per (b, h, 128-query tile): Q and dO stay; for every key
 //                     tile of the band S = Q K^T and dP = dO V^T, then dS (bf16, in TMEM)
 //                     and dQ += dS K.
@@ -44,25 +47,29 @@ __device__ __forceinline__ bool bwd_wait_warp(uint64_t* bar, uint32_t parity, ui
 constexpr int kBwdTcThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2..9 element-wise
 constexpr int kBwdTcEw = 256;       // element-wise threads: two warps per row quarter
 
-template <int D>
+template <int D, bool KV>
 struct BwdTcCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static constexpr int kBoxBytes = 128 * 128;
     static constexpr int kTileBytes = 128 * D * 2;
-    static constexpr int kStages = D == 128 ? 4 : 8;  // streamed tiles (Q/dO or K/V)
-    static constexpr int kFixOff = 0;                 // two resident tiles
-    static constexpr int kRingOff = 2 * kTileBytes;
+    // the key-tile kernel keeps K and V in shared memory; the query-tile kernel keeps Q and
+    // dO in TMEM and gives their room to the ring of streamed tiles (Q/dO or K/V)
+    static constexpr int kStages = KV ? (D == 128 ? 4 : 8) : (D == 128 ? 6 : 10);
+    static constexpr int kFixOff = 0;
+    static constexpr int kRingOff = KV ? 2 * kTileBytes : 0;
     static constexpr int kStatStages = 2;
     static constexpr int kStatBytes = 2 * 128 * 4;    // nlse2[128], delta[128]
     static constexpr int kStatOff = kRingOff + kStages * kTileBytes;
     static constexpr int kBarOff = kStatOff + kStatStages * kStatBytes;
-    // fix_full, ring_full[S], ring_empty[S], stat_full[2], stat_empty[2], s_full, p_full,
-    // o_final, drain, s_read
-    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 5;
+    // fix_full, ring_full[S], ring_empty[S], stat_full[2], stat_empty[2], s_full, s_read,
+    // dp_full[2], p_full[2], o_final, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 8;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 384;
+    // the query-tile kernel's resident Q and dO rows (A operands of S and dP)
+    static constexpr uint32_t kColQ = 384, kColDO = 448;
 };
 
 // delta_i = sum_d dout_i[d] out_i[d] (fp32) and nlse2_i = -lse_i * log2(e), one warp per row
@@ -165,17 +172,18 @@ __device__ __forceinline__ void bwd_store_row(uint32_t col, float a, __nv_bfloat
     }
 }
 
-// KV = true: bwd_kv_kernel (resident K, V; streamed Q, dO; dK, dV out).
-// KV = false: bwd_q_kernel (resident Q, dO; streamed K, V; dQ out).
+// KV = true: bwd_kv_kernel (resident K, V in shared memory; streamed Q, dO; dK, dV out).
+// KV = false: bwd_q_kernel (resident Q, dO in TMEM, read from rq, rdo; streamed K, V; dQ out).
 // Maps are 4-D {D, T, H, B} of contiguous [B,H,T,D] tensors. nlse2/delta: [B*H, Tpad].
 template <int D, bool KV>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __nv_bfloat16* __restrict__ rq, const __nv_bfloat16* __restrict__ rdo,
                   const float* __restrict__ nlse2, const float* __restrict__ delta, __nv_bfloat16* __restrict__ g1,
                   __nv_bfloat16* __restrict__ g2, int H, int T, int Tpad, int W, int n_t, float c, float c2,
                   uint64_t wait_limit_ns, int* status) {
-    using Cf = BwdTcCfg<D>;
+    using Cf = BwdTcCfg<D, KV>;
     constexpr int NS = Cf::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -187,10 +195,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     uint64_t* stat_full = ring_empty + NS;  // [2]
     uint64_t* stat_empty = stat_full + 2;   // [2]
     uint64_t* s_full = stat_empty + 2;
-    uint64_t* p_full = s_full + 1;
-    uint64_t* o_final = p_full + 1;
+    uint64_t* s_read = s_full + 1;   // the element-wise warps have read a tile's S
+    uint64_t* dp_full = s_read + 1;  // [2]: dP of one half of the tile's columns
+    uint64_t* p_full = dp_full + 2;  // [2]: P and dS of one half of the tile's columns
+    uint64_t* o_final = p_full + 2;
     uint64_t* drain = o_final + 1;
-    uint64_t* s_read = drain + 1;  // the element-wise warps have read S and dP of a tile
     const float* st_smem = reinterpret_cast<const float*>(smem + Cf::kStatOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cf::kMiscOff + 4);
@@ -213,7 +222,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     auto cls = [&](int yt) { return KV ? tile_class(T, W, 128, 128, yt, xt) : tile_class(T, W, 128, 128, xt, yt); };
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(fix_full, 1);
+        ptx::mbar_init(fix_full, KV ? 1 : kBwdTcEw);
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(ring_full + s, 1);
             ptx::mbar_init(ring_empty + s, 1);
@@ -223,10 +232,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             ptx::mbar_init(stat_empty + x, kBwdTcEw);
         }
         ptx::mbar_init(s_full, 1);
-        ptx::mbar_init(p_full, kBwdTcEw);
+        ptx::mbar_init(s_read, kBwdTcEw);
+        for (int x = 0; x < 2; ++x) {
+            ptx::mbar_init(dp_full + x, 1);
+            ptx::mbar_init(p_full + x, kBwdTcEw);
+        }
         ptx::mbar_init(o_final, 1);
         ptx::mbar_init(drain, 1);
-        ptx::mbar_init(s_read, kBwdTcEw);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -255,12 +267,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             const CUtensorMap* fb = KV ? &tm_v : &tm_do;
             const CUtensorMap* sa = KV ? &tm_q : &tm_k;   // streamed operands
             const CUtensorMap* sb = KV ? &tm_do : &tm_v;
-            ptx::mbar_arrive_expect_tx(fix_full, 2 * Cf::kTileBytes);
-            for (int x = 0; x < 2; ++x)
-                for (int cc = 0; cc < D / 64; ++cc)
-                    ptx::tma_load_4d(smem + Cf::kFixOff + x * Cf::kTileBytes + cc * Cf::kBoxBytes, x ? fb : fa,
-                                     fix_full, cc * 64, 128 * xt, h, b);
-            fix_issued = true;
+            if (KV) {
+                ptx::mbar_arrive_expect_tx(fix_full, 2 * Cf::kTileBytes);
+                for (int x = 0; x < 2; ++x)
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        ptx::tma_load_4d(smem + Cf::kFixOff + x * Cf::kTileBytes + cc * Cf::kBoxBytes, x ? fb : fa,
+                                         fix_full, cc * 64, 128 * xt, h, b);
+                fix_issued = true;
+            }
             for (int yt = lo; yt <= hi && ok; ++yt) {
                 if (cls(yt) == 0) continue;
                 for (int x = 0; x < 2 && ok; ++x) {
@@ -296,8 +310,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     } else if (warp == 1) {
         {
             // ---------------------------------------------------------------- MMA issuer
-            // (the whole warp runs this loop; its waits are warp-uniform, one lane issues)
+            // (the whole warp runs this loop; its waits are warp-uniform, one lane issues).
+            // A tile's 128 streamed columns are handled in two halves of 64: the element-wise
+            // warps turn half h of dP into P and dS, the gradient products of that half follow
+            // at once, and so does the next tile's dP for the same half (over the P and dS
+            // those products have just read), while the warps work on the other half.
             const uint32_t idesc_s = umma::idesc_bf16_f32(128, 128, 0);
+            const uint32_t idesc_dp = umma::idesc_bf16_f32(128, 64, 0);
             const uint32_t idesc_o = umma::idesc_bf16_f32(128, D, 1);
             const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
             const uint32_t lo_k = (uint32_t)umma::smem_desc(0, 16, 1024);
@@ -322,18 +341,29 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss_one(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k), desc_hi | ((a_lo + off) | lo_k),
-                                idesc_s, kk > 0 ? 1u : 0u);
+                    if (KV)
+                        ptx::mma_ss_one(tmem + Cf::kColS, desc_hi | ((fa_lo + off) | lo_k),
+                                        desc_hi | ((a_lo + off) | lo_k), idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_ts_one(tmem + Cf::kColS, tmem + Cf::kColQ + 8 * kk, desc_hi | ((a_lo + off) | lo_k),
+                                        idesc_s, kk > 0 ? 1u : 0u);
                 }
+                ptx::tc_commit_one(s_full);
             };
-            auto issue_dp = [&](uint32_t Lj) {
-                const uint32_t b_lo = ring_lo + ((Lj + 1) % NS) * kStageLo;
+            // dP of the streamed rows 64 hf .. 64 hf + 63 into TMEM columns 64 hf .. of the dP buffer
+            auto issue_dp = [&](uint32_t Lj, uint32_t hf) {
+                const uint32_t b_lo = ring_lo + ((Lj + 1) % NS) * kStageLo + hf * (64 * 128 >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * Cf::kBoxBytes + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss_one(tmem + Cf::kColDP, desc_hi | ((fb_lo + off) | lo_k), desc_hi | ((b_lo + off) | lo_k),
-                                idesc_s, kk > 0 ? 1u : 0u);
+                    if (KV)
+                        ptx::mma_ss_one(tmem + Cf::kColDP + 64 * hf, desc_hi | ((fb_lo + off) | lo_k),
+                                        desc_hi | ((b_lo + off) | lo_k), idesc_dp, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_ts_one(tmem + Cf::kColDP + 64 * hf, tmem + Cf::kColDO + 8 * kk,
+                                        desc_hi | ((b_lo + off) | lo_k), idesc_dp, kk > 0 ? 1u : 0u);
                 }
+                ptx::tc_commit_one(dp_full + hf);
             };
             uint32_t L = 0;
             int j = 0;  // visited tiles
@@ -342,12 +372,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             if (ok) {
                 ptx::tc_fence_after();
                 issue_s(0);
-                issue_dp(0);
-                ptx::tc_commit_one(s_full);
+                issue_dp(0, 0);
+                issue_dp(0, 1);
             }
             while (ok) {
                 const int ynext = next_visited(yt);
-                // the next tile's scores as soon as this tile's S and dP are in registers
+                // the next tile's scores as soon as this tile's S is in registers
                 ok = bwd_wait_warp(s_read, j & 1, wait_limit_ns, abort_flag);
                 if (ok && ynext <= hi) {
                     ok = wait_stage(L + 2);
@@ -356,38 +386,49 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                         issue_s(L + 2);
                     }
                 }
-                if (ok) ok = bwd_wait_warp(p_full, j & 1, wait_limit_ns, abort_flag);
-                if (!ok) break;
-                ptx::tc_fence_after();
                 const uint32_t sta = L % NS, stb = (L + 1) % NS;
                 const uint32_t a_lo = ring_lo + sta * kStageLo, b_lo = ring_lo + stb * kStageLo;
-                if (KV) {
-                    // dV += P^T dO (A = P^T, the +16 half of each dP chunk; B = dO);
-                    // dK += dS^T Q (A = dS^T, the first half; B = Q)
+                for (uint32_t hf = 0; hf < 2 && ok; ++hf) {
+                    ok = bwd_wait_warp(p_full + hf, j & 1, wait_limit_ns, abort_flag);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    if (KV) {
+                        // dV += P^T dO (A = P^T, the +16 half of each dP chunk; B = dO);
+                        // dK += dS^T Q (A = dS^T, the first half; B = Q)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk) + 16,
-                                    desc_hi | ((b_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = 4 * hf + k4;
+                            ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk) + 16,
+                                        desc_hi | ((b_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts_one(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
-                                    desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                } else {
-                    // dQ += dS K (A = dS in the dP columns, B = K)
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = 4 * hf + k4;
+                            ptx::mma_ts_one(tmem + Cf::kColB, tmem + Cf::kColDP + pp_pcol(kk),
+                                        desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    } else {
+                        // dQ += dS K (A = dS in the dP columns, B = K)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk),
-                                    desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = 4 * hf + k4;
+                            ptx::mma_ts_one(tmem + Cf::kColA, tmem + Cf::kColDP + pp_pcol(kk),
+                                        desc_hi | ((a_lo + kk * (2048 >> 4)) | lo_mn), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    if (hf == 1) {
+                        ptx::tc_commit_one(ring_empty + sta);
+                        ptx::tc_commit_one(ring_empty + stb);
+                    }
+                    // the next tile's dP for this half, after the products above read its P and dS
+                    if (ynext <= hi) {
+                        ok = wait_stage(L + 3);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        issue_dp(L + 2, hf);
+                    }
                 }
-                ptx::tc_commit_one(ring_empty + sta);
-                ptx::tc_commit_one(ring_empty + stb);
-                if (ynext > hi) break;
-                // the next tile's dP, over this tile's P and dS, after the products above read them
-                ok = wait_stage(L + 3);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                issue_dp(L + 2);
-                ptx::tc_commit_one(s_full);
+                if (!ok || ynext > hi) break;
                 L += 2;
                 ++j;
                 yt = ynext;
@@ -400,7 +441,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
     } else {
         // -------------------------------------------------------------------- element-wise
-        // warps 2..9: warp w serves TMEM lanes 32*(w%4).. and column chunks 2*half, 2*half+1
+        // warps 2..9: warp w serves TMEM lanes 32*(w%4).. and column chunks half, 2+half
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;  // the TMEM lane = this thread's resident row
@@ -410,6 +451,30 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         if (!KV) {
             my_nlse2 = nlse2[(int64_t)bh * Tpad + xr];  // -inf on padding rows: P = 0
             my_delta = delta[(int64_t)bh * Tpad + xr];
+            // this thread's half of its rows of q and dout (zero past T) into TMEM, where
+            // column c holds elements 2c and 2c+1: the A operands of S and dP
+            constexpr int HE = D / 2;
+            const bool live = xr < T;
+            const int64_t src = ((int64_t)bh * T + (live ? xr : 0)) * D + HE * half;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const uint4* p4 = reinterpret_cast<const uint4*>((x ? rdo : rq) + src);
+                uint32_t w[HE / 2];
+#pragma unroll
+                for (int t = 0; t < HE / 8; ++t) {
+                    const uint4 u = live ? p4[t] : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * t] = u.x;
+                    w[4 * t + 1] = u.y;
+                    w[4 * t + 2] = u.z;
+                    w[4 * t + 3] = u.w;
+                }
+                const uint32_t col = tl + (x ? Cf::kColDO : Cf::kColQ) + (HE / 2) * half;
+                if constexpr (D == 128) ptx::tmem_st32(col, w);
+                else ptx::tmem_st16(col, w);
+            }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(fix_full);
         }
         bool ok = true;
         int j = 0;
@@ -433,10 +498,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                 if (xr >= T) clo = chi + 1;
             }
             if (KV && xr >= T) clo = chi + 1;
-            // the scores first, so that the S columns can take the next tile's scores
+            // the scores first, so that the S columns can take the next tile's scores; this
+            // warp's chunks are half (columns 0..63) and 2 + half (columns 64..127)
             uint32_t sv[2][32];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) ptx::tmem_ld32(tl + Cf::kColS + 32 * (2 * half + x), sv[x]);
+            for (int x = 0; x < 2; ++x) ptx::tmem_ld32(tl + Cf::kColS + 32 * (2 * x + half), sv[x]);
             ptx::tmem_ld_wait();
 #pragma unroll
             for (int x = 0; x < 2; ++x) ptx::reg_fence(sv[x]);
@@ -444,7 +510,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
             ptx::mbar_arrive(s_read);
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
-                const int cc = 2 * half + x;
+                const int cc = 2 * x + half;
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(dp_full + x, j & 1, wait_limit_ns, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
                 const uint32_t dc = tl + Cf::kColDP + 32 * cc;
                 uint32_t dpv[32];
                 ptx::tmem_ld32(dc, dpv);
@@ -459,11 +530,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                     if (edge) bwd_chunk<false, true, false>(sv[x], dpv, dc, c2, nullptr, nullptr, my_nlse2, my_delta, cmin, cmax);
                     else bwd_chunk<false, false, false>(sv[x], dpv, dc, c2, nullptr, nullptr, my_nlse2, my_delta, cmin, cmax);
                 }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(p_full + x);
             }
-            ptx::tmem_st_wait();
-            ptx::tc_fence_before();
+            if (!ok) break;
             if (KV) ptx::mbar_arrive(stat_empty + (j & 1));
-            ptx::mbar_arrive(p_full);
             ++j;
         }
         if (ok) {

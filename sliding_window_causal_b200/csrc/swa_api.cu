@@ -98,10 +98,10 @@ cudaError_t set_pp_attrs(bool* regs_ok) {
 template <int D>
 cudaError_t set_bwd_tc_attrs() {
     cudaError_t e = cudaFuncSetAttribute(swa::bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         swa::BwdTcCfg<D>::kSmemBytes);
+                                         swa::BwdTcCfg<D, true>::kSmemBytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(swa::bwd_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 swa::BwdTcCfg<D>::kSmemBytes);
+                                 swa::BwdTcCfg<D, false>::kSmemBytes);
     return e;
 }
 
@@ -803,18 +803,18 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
         auto* gk = static_cast<__nv_bfloat16*>(dk);
         auto* gv = static_cast<__nv_bfloat16*>(dv);
         if (D == 128) {
-            swa::bwd_tc_kernel<128, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+            swa::bwd_tc_kernel<128, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128, true>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
-            swa::bwd_tc_kernel<128, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+            swa::bwd_tc_kernel<128, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128, false>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
         } else {
-            swa::bwd_tc_kernel<64, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+            swa::bwd_tc_kernel<64, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64, true>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
-            swa::bwd_tc_kernel<64, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+            swa::bwd_tc_kernel<64, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64, false>::kSmemBytes, s>>>(
+                mq, mk, mv, mdo, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
                 ds->status);
         }
         cudaError_t e = cudaGetLastError();

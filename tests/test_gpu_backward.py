@@ -47,7 +47,9 @@ def test_backward_fp32(B, H, T, D, W):
 
 
 @pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 300, 64, 77), (1, 2, 257, 128, 128), (2, 1, 129, 128, 1000),
-                                       (1, 1, 200, 32, 50), (2, 2, 640, 128, 1), (1, 2, 1000, 64, 300)])
+                                       (1, 1, 200, 32, 50), (2, 2, 640, 128, 1), (1, 2, 1000, 64, 300),
+                                       (1, 1, 65, 128, 64), (1, 2, 191, 64, 63), (1, 1, 384, 128, 65),
+                                       (1, 1, 2048, 64, 700)])
 def test_backward_bf16(B, H, T, D, W):
     check(B, H, T, D, W, torch.bfloat16, 23 + T + W)
 
