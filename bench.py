@@ -61,11 +61,9 @@ def _scaled(kind, captured):
 
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
-    "prefill": {"bytes": 532.1e6 + 112.9e6, "sources": "363d93e3c1503ea4"},
-    # decode.cuh is unchanged since the capture; ptx.cuh has since gained helpers the
-    # decode kernel does not use
-    "decode": {"bytes": _scaled("decode", 951.0e6 + 3.5e6), "sources": "69ace3889ab1351e"},
-    "chunk": {"bytes": _scaled("chunk", 1105.6e6 + 17.7e6), "sources": "d2e5b2317b60e3ce"},
+    "prefill": {"bytes": 534.6e6 + 112.9e6, "sources": "0126a7cf0c675360"},
+    "decode": {"bytes": _scaled("decode", 951.0e6 + 3.9e6), "sources": "be9af298ce410eec"},
+    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 18.0e6), "sources": "481afa7276ce1753"},
 }
 
 
