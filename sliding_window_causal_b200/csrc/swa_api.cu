@@ -22,6 +22,7 @@
 #include "chunk.cuh"
 #include "decode.cuh"
 #include "plan.h"
+#include "prefill_narrow.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_pp.cuh"
 #include "weights.cuh"
@@ -341,6 +342,8 @@ int check_forward(const char* fn, const void* q, const void* k, const void* v, c
                                 "has stride %lld",
                                 fn, a, (long long)st[a][x]);
         if ((T + 127) / 128 * (B * H) > INT32_MAX) return fail(SWA_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+        if ((W < T ? W : T) <= swa::kNarrowMaxW && (T + swa::kNarrowRows - 1) / swa::kNarrowRows * (B * H) > INT32_MAX)
+            return fail(SWA_ERR_UNSUPPORTED, "%s: too many row blocks", fn);
     } else {
         if (D > 4096) return fail(SWA_ERR_UNSUPPORTED, "%s: fp32 supports D <= 4096", fn);
         if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
@@ -367,7 +370,31 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
 
-    if (dtype == SWA_BF16) {
+    if (dtype == SWA_BF16 && Wi <= swa::kNarrowMaxW) {
+        // bands of a few keys: bound by HBM, served on the CUDA cores without the tensor-core
+        // pipeline's fill and drain
+        const int64_t BH = B * H;
+        const int n_rb = (int)((T + swa::kNarrowRows - 1) / swa::kNarrowRows);
+        swa::Strides sx;
+        for (int x = 0; x < 3; ++x) {
+            sx.q[x] = st[0][x];
+            sx.k[x] = st[1][x];
+            sx.v[x] = st[2][x];
+            sx.o[x] = st[3][x];
+        }
+        const float scale_log2 = (float)(1.4426950408889634 * scale);
+        const auto* qb = static_cast<const __nv_bfloat16*>(q);
+        const auto* kb = static_cast<const __nv_bfloat16*>(k);
+        const auto* vb = static_cast<const __nv_bfloat16*>(v);
+        auto* ob = static_cast<__nv_bfloat16*>(out);
+        const unsigned grid = (unsigned)(BH * n_rb);
+        if (D == 128)
+            swa::prefill_narrow_kernel<128><<<grid, swa::kNarrowWarps * 32, 0, s>>>(qb, kb, vb, ob, sx, lse, (int)H,
+                                                                                 (int)T, Wi, scale_log2, n_rb);
+        else
+            swa::prefill_narrow_kernel<64><<<grid, swa::kNarrowWarps * 32, 0, s>>>(qb, kb, vb, ob, sx, lse, (int)H,
+                                                                                (int)T, Wi, scale_log2, n_rb);
+    } else if (dtype == SWA_BF16) {
         const int64_t BH = B * H;
         const int n_qt = (int)((T + 127) / 128);
         CUtensorMap mq, mk, mv;

@@ -88,9 +88,11 @@ def test_backward_deterministic():
     assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
-def test_lse_matches_oracle_weights():
-    """forward_lse's lse is log of the sum of exp(scaled score) over each band."""
-    B, H, T, D, W = 1, 2, 200, 64, 50
+@pytest.mark.parametrize("D,W", [(64, 50), (128, 6)])
+def test_lse_matches_oracle_weights(D, W):
+    """forward_lse's lse is log of the sum of exp(scaled score) over each band (W = 6:
+    the bf16 CUDA-core kernel for short bands)."""
+    B, H, T = 1, 2, 200
     for dtype in (torch.float32, torch.bfloat16):
         q, k, v = inputs.prefill_inputs(B, H, T, D, dtype, 47)
         out, lse = swa.forward_lse(q.to(DEV), k.to(DEV), v.to(DEV), W)

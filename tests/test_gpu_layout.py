@@ -33,6 +33,8 @@ LAYOUT_SHAPES = [
     (1, 4, 300, 64, 77, torch.bfloat16), (2, 3, 1000, 128, 129, torch.bfloat16),
     (1, 2, 777, 128, 5000, torch.bfloat16), (1, 8, 512, 64, 128, torch.bfloat16),
     (2, 3, 50, 4, 6, torch.float32), (1, 2, 257, 33, 40, torch.float32),
+    # short bands: the bf16 CUDA-core kernel reads the same strides
+    (2, 3, 200, 128, 5, torch.bfloat16), (1, 4, 77, 64, 1, torch.bfloat16),
 ]
 
 

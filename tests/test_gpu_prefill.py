@@ -49,6 +49,11 @@ BF16_SHAPES = [
     # either side of the band length (1024 keys) where the kernel moves from two MMA
     # issuers to one
     (1, 2, 3000, 128, 1024), (1, 2, 3000, 128, 1025), (1, 2, 2000, 64, 1500),
+    # bands of at most 7 keys take the CUDA-core kernel (32 rows a CTA): ragged and short
+    # T, band lengths up to 7, and 8 and 9, the first bands of the tensor-core kernel
+    (2, 2, 333, 128, 8), (1, 3, 95, 64, 5), (1, 2, 33, 128, 4), (1, 1, 7, 128, 8),
+    (2, 1, 500, 64, 7), (1, 2, 64, 128, 6), (1, 2, 300, 128, 9), (1, 1, 31, 64, 8),
+    (1, 2, 200, 64, 7),
 ]
 
 
