@@ -211,8 +211,8 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
 // m is the row's reference maximum (-inf until the row meets its first in-band key). A
 // row that sees its first keys takes the tile maximum; a row whose maximum exceeds m by
 // more than the rescale threshold moves m up by the integer k = ceil(excess) and scales
-// O and l by 2^-k (exact). The row sum adds the weights exactly as written, so O is
-// normalised by the weights the MMAs multiply by.
+// O and l by 2^-k (exact; zero when k > 126, where they are negligible). The row sum adds
+// the weights exactly as written, so O is normalised by the weights the MMAs multiply by.
 // MASK: 0 every key of the tile is in the row's band; 1 only columns cmin..cmax are; 2
 // columns cmin..cmax and cmin2..cmax2 are. before_rescale() runs (warp-uniformly) before O
 // is rescaled, for callers whose last P.V product may still be in flight. after_part(s)
@@ -267,8 +267,11 @@ __device__ __forceinline__ float pp_tile(uint32_t scol, uint32_t ocol, float sca
     const float tm = ptx::max3(ptx::max3(q[0], q[1], q[2]), ptx::max3(q[3], q[4], q[5]), fmaxf(q[6], q[7])) * scale_log2;
     const bool need = m != -INFINITY && tm > m + kPPRescaleThreshold;
     if (__any_sync(0xffffffffu, need)) {
-        const int k = need ? min(126, (int)ceilf(tm - m)) : 0;
-        const float f = pp_pow2_neg(k);
+        // k = ceil(excess) in full, so that no weight of this tile exceeds 2^0 (a capped k
+        // would leave exp2 of the rest to overflow); beyond 2^-126 the old O and l are below
+        // fp32's normal range relative to the new maximum and are dropped (f = 0)
+        const int k = need ? (int)fminf(ceilf(tm - m), 1048576.0f) : 0;
+        const float f = k > 126 ? 0.f : pp_pow2_neg(k);
         before_rescale();
         __syncwarp();
         pp_rescale<D, PRECISE>(ocol, scol, 0, f);

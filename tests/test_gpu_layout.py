@@ -12,7 +12,7 @@ import torch
 import oracle
 import sliding_window_causal_b200 as swa
 from sliding_window_causal_b200 import _native, inputs
-from gpu_util import TOL, f64, max_err
+from gpu_util import TOL, f64, max_err, sharp_inputs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -195,25 +195,6 @@ def test_mistral_bthd_full_size_equals_contiguous():
     swa.device_status()
     assert a.stride() == dq.stride()
     assert torch.equal(a.contiguous(), b)
-
-
-def sharp_inputs(B, H, T, D, seed, kind):
-    """Inputs whose rows are dominated by a few keys: "growing" (scores rise along the
-    sequence, so the newest keys dominate), "falling" (they fall, so the oldest keys of
-    each band dominate) or "spikes" (a few keys with large scores anywhere). v ~ N(0,1)."""
-    gen = torch.Generator().manual_seed(seed)
-    q = torch.ones(B, H, T, D)
-    t = torch.arange(T, dtype=torch.float32)
-    if kind == "growing":
-        base = 0.05 * t
-    elif kind == "falling":
-        base = -0.05 * t
-    else:
-        base = torch.zeros(T)
-        base[torch.randint(0, T, (T // 50,), generator=gen)] = 1.0
-    k = base[None, None, :, None].expand(B, H, T, D).clone() + 0.01 * torch.randn(B, H, T, D, generator=gen)
-    v = torch.randn(B, H, T, D, generator=gen)
-    return tuple(x.to(torch.bfloat16) for x in (q, k, v))
 
 
 @pytest.mark.parametrize("kind", ["growing", "falling", "spikes"])

@@ -183,6 +183,24 @@ def test_timeout_path_reports_and_recovers():
 # Every element of the full-size workloads is compared in test_gpu_fullsize.py; here the
 # properties that hold at any size, over every output of the Mistral-shaped workload.
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_score_jump_in_a_later_key_tile(D):
+    """One key whose scaled score exceeds every earlier key of the band by far more than
+    fp32's exponent range (about 650 in log2 units): the rows whose band holds it, and
+    which met ordinary keys in earlier key tiles first, must come out as that key's v, as
+    the oracle's max-subtracted softmax gives, not overflow."""
+    B, H, T, W = 1, 2, 1000, 600
+    q, k, v = inputs.prefill_inputs(B, H, T, D, torch.bfloat16, 301 + D)
+    q = torch.ones_like(q)
+    k = (0.01 * k.float()).to(torch.bfloat16)
+    k[:, :, 300] = 40.0 * 128.0 / D  # q . k_300 = 5120: 653 log2 units after the scale at D = 128
+    out = run(q, k, v, W)
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    err = max_err(out, ref)
+    assert err <= TOL[torch.bfloat16], f"max err {err}"
+    assert torch.equal(out.cpu()[:, :, 300:900], v[:, :, 300:301].expand(B, H, 600, D))
+
+
 def test_mistral_shaped_properties():
     wl = inputs.MISTRAL
     q, k, v = inputs.for_workload(wl)
