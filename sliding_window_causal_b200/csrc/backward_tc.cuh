@@ -92,8 +92,21 @@ __global__ void __launch_bounds__(256)
     }
     const int64_t src = (bh * T + i) * D;
     float acc = 0.f;
-    for (int d = lane; d < D; d += 32)
-        acc = fmaf(__bfloat162float(dout[src + d]), __bfloat162float(out[src + d]), acc);
+    // D/32 consecutive elements a lane (D is 64 or 128, rows 16-byte aligned): one 4- or
+    // 8-byte load of each tensor, so a warp reads each row in one coalesced pass
+    if (D == 128) {
+        const uint2 a = *reinterpret_cast<const uint2*>(dout + src + 4 * lane);
+        const uint2 o = *reinterpret_cast<const uint2*>(out + src + 4 * lane);
+        acc = ptx::bf16lo_f32(a.x) * ptx::bf16lo_f32(o.x);
+        acc = fmaf(ptx::bf16hi_f32(a.x), ptx::bf16hi_f32(o.x), acc);
+        acc = fmaf(ptx::bf16lo_f32(a.y), ptx::bf16lo_f32(o.y), acc);
+        acc = fmaf(ptx::bf16hi_f32(a.y), ptx::bf16hi_f32(o.y), acc);
+    } else {
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(dout + src + 2 * lane);
+        const uint32_t o = *reinterpret_cast<const uint32_t*>(out + src + 2 * lane);
+        acc = ptx::bf16lo_f32(a) * ptx::bf16lo_f32(o);
+        acc = fmaf(ptx::bf16hi_f32(a), ptx::bf16hi_f32(o), acc);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) {
