@@ -129,15 +129,24 @@ struct PPItem {
     bool hasB;
 };
 
-__device__ __forceinline__ PPItem pp_decode(int u, int BH, int H, int n_qt, int T, int W) {
+// single: each item is one query tile (used when a problem has fewer pairs of query tiles
+// than the grid has SMs, so that more CTAs work); item u is tile u % n_qt of (b, h) u / n_qt.
+__device__ __forceinline__ PPItem pp_decode(int u, int BH, int H, int n_qt, int T, int W, bool single) {
     PPItem it;
     int bh, p;
-    prefill_item<int>(u, BH, n_qt, W, &bh, &p);  // u is in range: pp_item checked it
+    if (single) {
+        bh = u / n_qt;
+        it.qt[0] = u - bh * n_qt;
+        it.qt[1] = it.qt[0] + 1;
+        it.hasB = false;
+    } else {
+        prefill_item<int>(u, BH, n_qt, W, &bh, &p);  // u is in range: pp_item checked it
+        it.qt[0] = 2 * p;
+        it.qt[1] = 2 * p + 1;
+        it.hasB = it.qt[1] < n_qt;
+    }
     it.b = bh / H;
     it.h = bh - it.b * H;
-    it.qt[0] = 2 * p;
-    it.qt[1] = 2 * p + 1;
-    it.hasB = it.qt[1] < n_qt;
     int64_t f, l;
     kv_tile_range(T, W, 128, 128, it.qt[0], &f, &l);
     it.f[0] = (int)f;
@@ -468,8 +477,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     uint4* fix_slot = reinterpret_cast<uint4*>(smem + C::kFixOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = ((n_qt + 1) >> 1) * BH;
     const int G = gridDim.x, g = blockIdx.x;
+    // pairs of query tiles as items, or single tiles when there are fewer pairs than CTAs
+    // (the host then sizes the grid by the single tiles)
+    const int n_pairs = ((n_qt + 1) >> 1) * BH;
+    const bool single = G > n_pairs;
+    const int n_items = single ? n_qt * BH : n_pairs;
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
@@ -521,7 +534,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
                 if (u < 0) break;
-                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W, single);
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (!ok || (x == 1 && !it.hasB)) break;
@@ -579,7 +592,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
                 if (u < 0) break;
-                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W, single);
                 const int nx = it.hasB ? 2 : 1;
                 const bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
 #pragma unroll
@@ -693,7 +706,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int r = 0; ok; ++r) {
                 const int u = pp_item(r, g, G, n_items);
                 if (u < 0) break;
-                const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
+                const PPItem it = pp_decode(u, BH, H, n_qt, T, W, single);
                 const bool mine = x == 0 || it.hasB;
                 const int f = it.f[x], l = it.l[x];
                 const bool prec = pp_precise(it.qt[x], W);
@@ -827,7 +840,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int rr = 0; ok; ++rr) {
             const int u = pp_item(rr, g, G, n_items);
             if (u < 0) break;
-            const PPItem it = pp_decode(u, BH, H, n_qt, T, W);
+            const PPItem it = pp_decode(u, BH, H, n_qt, T, W, single);
             if (x == 1 && !it.hasB) continue;
             const int qt = x ? it.qt[1] : it.qt[0];
             const int fx = x ? it.f[1] : it.f[0];

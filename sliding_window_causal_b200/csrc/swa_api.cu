@@ -406,7 +406,10 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
         if (!ds->pp_regs_ok)
             return fail(SWA_ERR_UNSUPPORTED, "%s: prefill kernel was not compiled with %d registers per thread",
                         fn, swa::kPPLaunchRegs);
-        const int64_t n_items = (int64_t)((n_qt + 1) / 2) * BH;
+        // pairs of query tiles as work items; single tiles when there are fewer pairs than SMs
+        // (the kernel tells the two apart by the grid size)
+        const int64_t n_pairs = (int64_t)((n_qt + 1) / 2) * BH;
+        const int64_t n_items = n_pairs < ds->num_sms ? (int64_t)n_qt * BH : n_pairs;
         const unsigned G = (unsigned)(n_items < ds->num_sms ? n_items : ds->num_sms);
         auto* ob = static_cast<__nv_bfloat16*>(out);
         swa::PPRaw raw;
