@@ -48,7 +48,7 @@ struct ChunkCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static constexpr int kBoxBytes = 128 * 128;         // 128 rows x 64 bf16
     static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile of Q, K or V
-    static constexpr int kStages = D == 128 ? 5 : 10;   // unified K/V ring
+    static constexpr int kStages = D == 128 ? 6 : 12;   // unified K/V ring
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = kTileBytes;
     static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
