@@ -4,7 +4,10 @@ import torch
 
 # Tolerances on max |GPU - float64 oracle| over compared elements: fp32 in/out 1e-5,
 # bf16 in/out with fp32 accumulation 1e-2 (the oracle runs on the same bf16-rounded
-# inputs, widened exactly to float64).
+# inputs, widened exactly to float64). A bf16 output cannot come closer to a real number
+# than half the bf16 spacing there, which exceeds 1e-2 from magnitude 4 on (spacing 2^-5);
+# so a bf16 element that is one of the two bf16 values bracketing the oracle's value also
+# passes. Below magnitude 4 some bf16 value always lies within 1e-2, and the bar is 1e-2.
 TOL = {torch.float32: 1e-5, torch.bfloat16: 1e-2}
 
 
@@ -12,8 +15,24 @@ def f64(t):
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+def bf16_bracket(r):
+    """The largest and smallest bf16 values with lo <= r <= hi (equal when r is one),
+    for finite float64 r in bf16's normal range: bf16 has 8 significand bits, so its
+    spacing at |r| in [2^e, 2^(e+1)) is 2^(e-7)."""
+    a = np.abs(r)
+    ulp = np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7)
+    return np.floor(r / ulp) * ulp, np.ceil(r / ulp) * ulp
+
+
 def max_err(gpu_out, ref):
-    return float(np.abs(f64(gpu_out) - ref).max()) if ref.size else 0.0
+    if not ref.size:
+        return 0.0
+    g = f64(gpu_out)
+    e = np.abs(g - ref)
+    if gpu_out.dtype == torch.bfloat16:
+        lo, hi = bf16_bracket(ref)
+        e = np.where((e > TOL[torch.bfloat16]) & ((g == lo) | (g == hi)), 0.0, e)
+    return float(e.max())
 
 
 def sharp_inputs(B, H, T, D, seed, kind):

@@ -201,6 +201,19 @@ def test_score_jump_in_a_later_key_tile(D):
     assert torch.equal(out.cpu()[:, :, 300:900], v[:, :, 300:301].expand(B, H, 600, D))
 
 
+@pytest.mark.parametrize("H", [147, 148, 149])
+def test_work_items_either_side_of_the_sm_count(H):
+    """Fewer pairs of query tiles than SMs make each work item a single query tile; at or
+    above the SM count (148 on a B200) items are pairs. Two tiles per head (T = 256), so
+    H is the number of pairs: every row against the oracle on either side of the switch."""
+    B, T, D, W = 1, 256, 64, 100
+    q, k, v = inputs.prefill_inputs(B, H, T, D, torch.bfloat16, 400 + H)
+    out = run(q, k, v, W)
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    err = max_err(out, ref)
+    assert err <= TOL[torch.bfloat16], f"H {H}: max err {err}"
+
+
 def test_mistral_shaped_properties():
     wl = inputs.MISTRAL
     q, k, v = inputs.for_workload(wl)
