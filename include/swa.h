@@ -383,6 +383,20 @@ int swa_prefill_work_item(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W,
                           int64_t* h, int64_t* pair);
 
 /*
+ * swa_backward_cta_tile: the resident tile of the u-th CTA of the tensor-core backward
+ * (bf16, D 64 or 128) for sizes B, H, T and window W. kv != 0: the key-tile kernel
+ * (dK, dV), whose key tile kt meets min(n_t - kt, a + 1) query tiles; kv == 0: the
+ * query-tile kernel (dQ), whose query tile qt meets min(qt, a) + 1 key tiles; n_t =
+ * ceil(T/128) and a = ceil((min(W,T) - 1)/128). CTAs 0 .. B*H*n_t - 1 cover every
+ * (b, h, tile) once: first the tiles that meet a + 1 tiles, head after head, then the
+ * others heaviest first, head-minor, so that the last CTAs to start are the lightest.
+ * Writes *b, *h, *tile and returns 0, or returns -1 for invalid arguments (B, H, T or
+ * W < 1, u out of range, null pointers).
+ */
+int swa_backward_cta_tile(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W, int kv, int64_t* b,
+                          int64_t* h, int64_t* tile);
+
+/*
  * swa_decode_valid_slots: number n of ring slots that hold in-window positions for a
  * stream at position pos: n = min(pos + 1, W); the valid slots are 0 .. n-1.
  * Returns -1 if pos < 0 or W < 1.

@@ -347,6 +347,15 @@ def work_item(u, B, H, T, W):
     return None if rc != 0 else (b.value, h.value, p.value)
 
 
+def backward_cta_tile(u, B, H, T, W, kv):
+    """(b, h, tile) of the tensor-core backward's u-th CTA (see swa_backward_cta_tile): a
+    key tile when kv, else a query tile; None for invalid arguments."""
+    b, h, t = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    rc = _native.lib().swa_backward_cta_tile(u, B, H, T, W, 1 if kv else 0, ctypes.byref(b), ctypes.byref(h),
+                                             ctypes.byref(t))
+    return None if rc != 0 else (b.value, h.value, t.value)
+
+
 def valid_slots(pos, W):
     """Number of valid ring slots (slots 0..n-1) for a stream at position pos."""
     return _native.lib().swa_decode_valid_slots(pos, W)

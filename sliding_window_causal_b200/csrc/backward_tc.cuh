@@ -218,8 +218,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cf::kMiscOff + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x / n_t;
-    const int xt = blockIdx.x - bh * n_t;  // the resident tile: key tile (KV) or query tile
+    int bh, xt;  // the resident tile: key tile (KV) or query tile
+    bwd_cta_tile<int>((int)blockIdx.x, (int)gridDim.x / n_t, n_t, W, KV, &bh, &xt);
+    // The query-tile kernel follows this one as a programmatic dependent launch: it reads
+    // nothing this kernel writes, so its CTAs may take the SMs this grid's last CTAs leave.
+    if (KV) ptx::launch_dependents();
     const int b = bh / H, h = bh - b * H;
     // the streamed tiles that meet the band: query tiles xt .. (KV), or key tiles (Q)
     int lo, hi;
@@ -599,6 +602,9 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, Cf::kTmemCols);
     }
+    // The query-tile grid ends only after the key-tile grid it may overlap, so that the
+    // stream's next work sees dK and dV as well as dQ.
+    if (!KV) ptx::grid_dependency_wait();
 }
 
 }  // namespace swa

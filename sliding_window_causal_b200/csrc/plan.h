@@ -92,6 +92,35 @@ SWA_HD bool prefill_item(I u, I BH, I n_qt, I W, I* bh, I* pair) {
     return true;
 }
 
+// CTAs of the tensor-core backward: one per (bh, resident 128-row tile), BH * n_t in all;
+// the resident tile is a key tile (kv) or a query tile. With a = ceil((W - 1) / 128), key
+// tile kt streams the min(n_t - kt, a + 1) query tiles that meet its band (falling with
+// kt) and query tile qt the min(qt, a) + 1 key tiles of its band (rising with qt), so the
+// tiles that stream a + 1 tiles (full) are the first n_t - a key tiles or the last
+// n_t - a query tiles. CTA u is:
+//  - first the full tiles, head after head, those of a head in order: the CTAs at work
+//    at one time stream the tiles of a few heads, which stay in L2;
+//  - then the others heaviest first, head-minor, so that the last CTAs to start are the
+//    lightest and the SMs finish together.
+// W is the window clamped to T. Returns false if u is out of range.
+template <typename I>
+SWA_HD bool bwd_cta_tile(I u, I BH, I n_t, I W, bool kv, I* bh, I* xt) {
+    if (u < 0 || BH < 1 || n_t < 1 || W < 1 || u >= BH * n_t) return false;
+    const I a = (W + 126) / 128;
+    const I np = a < n_t ? a : n_t;  // tiles that stream fewer than a + 1 tiles
+    const I nf = n_t - np;
+    if (u < BH * nf) {
+        *bh = u / nf;
+        const I r = u % nf;
+        *xt = kv ? r : np + r;
+        return true;
+    }
+    const I v = u - BH * nf, r = v / BH;  // r = 0: the heaviest of the others
+    *bh = v % BH;
+    *xt = kv ? nf + r : np - 1 - r;
+    return true;
+}
+
 SWA_HD int64_t decode_valid_slots(int64_t pos, int64_t W) {
     return pos + 1 < W ? pos + 1 : W;
 }

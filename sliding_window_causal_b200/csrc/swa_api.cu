@@ -518,6 +518,17 @@ int swa_prefill_work_item(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W,
     return 0;
 }
 
+int swa_backward_cta_tile(int64_t u, int64_t B, int64_t H, int64_t T, int64_t W, int kv, int64_t* b, int64_t* h,
+                          int64_t* tile) {
+    if (B < 1 || H < 1 || T < 1 || W < 1 || !b || !h || !tile || B > INT32_MAX || H > INT32_MAX || T > INT32_MAX)
+        return -1;
+    int64_t bh;
+    if (!swa::bwd_cta_tile<int64_t>(u, B * H, (T + 127) / 128, W < T ? W : T, kv != 0, &bh, tile)) return -1;
+    *b = bh / H;
+    *h = bh % H;
+    return 0;
+}
+
 int64_t swa_decode_valid_slots(int64_t pos, int64_t W) {
     if (pos < 0 || W < 1) return -1;
     return swa::decode_valid_slots(pos, W);
@@ -832,22 +843,40 @@ int swa_backward(const void* q, const void* k, const void* v, const void* out, c
         auto* gq = static_cast<__nv_bfloat16*>(dq);
         auto* gk = static_cast<__nv_bfloat16*>(dk);
         auto* gv = static_cast<__nv_bfloat16*>(dv);
+        // The key-tile kernel, then the query-tile kernel as its programmatic dependent:
+        // the two share no output, so the second may start on the SMs the first one's
+        // last CTAs free (it waits for the first grid before it ends).
+        const auto* rq = static_cast<const __nv_bfloat16*>(q);
+        const auto* rdo = static_cast<const __nv_bfloat16*>(dout);
+        const uint64_t lim = wait_limit();
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t qc = {};
+        qc.gridDim = dim3(grid);
+        qc.blockDim = dim3(swa::kBwdTcThreads);
+        qc.stream = s;
+        qc.attrs = pdl;
+        qc.numAttrs = 1;
+        cudaError_t e;
         if (D == 128) {
             swa::bwd_tc_kernel<128, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128, true>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, lim,
                 ds->status);
-            swa::bwd_tc_kernel<128, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<128, false>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
-                ds->status);
+            qc.dynamicSmemBytes = swa::BwdTcCfg<128, false>::kSmemBytes;
+            e = cudaLaunchKernelEx(&qc, swa::bwd_tc_kernel<128, false>, mq, mk, mv, mdo, rq, rdo, (const float*)nlse2,
+                                   (const float*)delta, gq, (__nv_bfloat16*)nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t,
+                                   c, c2, lim, ds->status);
         } else {
             swa::bwd_tc_kernel<64, true><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64, true>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
+                mq, mk, mv, mdo, nullptr, nullptr, nlse2, delta, gk, gv, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, lim,
                 ds->status);
-            swa::bwd_tc_kernel<64, false><<<grid, swa::kBwdTcThreads, swa::BwdTcCfg<64, false>::kSmemBytes, s>>>(
-                mq, mk, mv, mdo, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), nlse2, delta, gq, nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t, c, c2, wait_limit(),
-                ds->status);
+            qc.dynamicSmemBytes = swa::BwdTcCfg<64, false>::kSmemBytes;
+            e = cudaLaunchKernelEx(&qc, swa::bwd_tc_kernel<64, false>, mq, mk, mv, mdo, rq, rdo, (const float*)nlse2,
+                                   (const float*)delta, gq, (__nv_bfloat16*)nullptr, (int)H, (int)T, (int)Tpad, Wi, n_t,
+                                   c, c2, lim, ds->status);
         }
-        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "swa_backward launch");
         return success();
     }

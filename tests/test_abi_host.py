@@ -1,6 +1,7 @@
 """C-ABI library on the CPU: it loads, exports every symbol include/swa.h declares, and
 its host-side work planning (tile classification, ring slots, decode splits) is
 bit-exact against brute-force enumeration. No GPU compute is called here."""
+import heapq
 import itertools
 import os
 import re
@@ -139,6 +140,52 @@ def test_work_item_rejects_bad_args():
     assert swa.work_item(0, 0, 1, 10, 3) is None
     assert swa.work_item(0, 1, 1, 0, 3) is None
     assert swa.work_item(0, 1, 1, 10, 0) is None
+
+
+def _streamed_tiles(T, W, tile, kv):
+    """Tiles the backward streams past a resident tile, by enumeration: the query tiles
+    that visit key tile `tile` (kv), or the key tiles that query tile `tile` visits."""
+    n = (T + 127) // 128
+    if kv:
+        return sum(1 for qt in range(n) if swa.tile_class(T, W, 128, 128, qt, tile) > 0)
+    return sum(1 for kt in range(n) if swa.tile_class(T, W, 128, 128, tile, kt) > 0)
+
+
+@pytest.mark.parametrize("kv", [True, False])
+@pytest.mark.parametrize("B,H,T,W", [(1, 32, 16384, 4096), (2, 16, 8192, 1), (2, 16, 8192, 1024),
+                                     (2, 16, 8192, 8192), (1, 8, 512, 128), (1, 3, 1000, 129),
+                                     (2, 3, 1300, 5000), (1, 2, 129, 64), (3, 1, 640, 300), (1, 1, 100, 7)])
+def test_backward_ctas_cover_every_tile_once_lightest_last(B, H, T, W, kv):
+    """The backward's CTAs are a permutation of all (b, h, tile); the tiles that stream the
+    most tiles come first, head after head and in order within a head; the rest follow
+    with non-increasing work; and CTAs dealt in that order to whichever of 148 SMs is free
+    first (a fixed cost of 1.5 tiles each) finish within 2 % of the mean."""
+    n_t = (T + 127) // 128
+    n = B * H * n_t
+    ctas = [swa.backward_cta_tile(u, B, H, T, W, kv) for u in range(n)]
+    assert sorted(ctas) == [(b, h, t) for b in range(B) for h in range(H) for t in range(n_t)]
+    assert swa.backward_cta_tile(n, B, H, T, W, kv) is None and swa.backward_cta_tile(-1, B, H, T, W, kv) is None
+    work = {t: _streamed_tiles(T, W, t, kv) for t in range(n_t)}
+    top = max(work.values())
+    nf = next((u for u, c in enumerate(ctas) if work[c[2]] != top), n)
+    assert all(work[t] != top for (_, _, t) in ctas[nf:]) or nf == 0, "the heaviest tiles come first"
+    head_order = [(b * H + h, t) for (b, h, t) in ctas[:nf]]
+    assert head_order == sorted(head_order), "head after head, tiles in order"
+    rest = [work[t] for (_, _, t) in ctas[nf:]]
+    assert rest == sorted(rest, reverse=True), "the rest heaviest first"
+    if n >= 8 * 148:
+        free = [0.0] * 148
+        heapq.heapify(free)
+        for (_, _, t) in ctas:
+            heapq.heappush(free, heapq.heappop(free) + work[t] + 1.5)
+        mean = sum(work[t] + 1.5 for (_, _, t) in ctas) / 148
+        assert max(free) <= 1.02 * mean
+
+
+def test_backward_cta_tile_rejects_bad_args():
+    assert swa.backward_cta_tile(0, 0, 1, 10, 3, True) is None
+    assert swa.backward_cta_tile(0, 1, 1, 0, 3, False) is None
+    assert swa.backward_cta_tile(0, 1, 1, 10, 0, True) is None
 
 
 def test_valid_slots_match_ring_enumeration():
