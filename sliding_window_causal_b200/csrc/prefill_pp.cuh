@@ -98,18 +98,23 @@ struct PPRaw {
     int64_t sq[3], sk[3], sv[3];
 };
 
-template <int D>
+// TWO (two MMA issuers, short bands): two sets of Q_A, Q_B buffers, so that the producer
+// loads the next item's Q while the current item still uses its own, and a shallower ring.
+// An item of a short band streams few key tiles, so its start (Q and the first key tile
+// arriving) weighs more than the ring depth within it.
+template <int D, bool TWO = false>
 struct PPCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 64 bf16
     static constexpr int kTileBytes = 128 * D * 2;     // one 128-row tile of Q, K or V
-    static constexpr int kStages = D == 128 ? 5 : 12;  // unified K/V ring
-    static constexpr int kQOff = 0;                    // Q_A, Q_B
-    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kQSets = TWO ? 2 : 1;         // sets of Q_A, Q_B
+    static constexpr int kStages = D == 128 ? (TWO ? 3 : 5) : (TWO ? 10 : 12);  // unified K/V ring
+    static constexpr int kQOff = 0;                    // Q set s, tile x at (2s + x) tiles
+    static constexpr int kRingOff = 2 * kQSets * kTileBytes;
     static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-    // q_full[2], q_empty[2], ring_full[S], ring_empty[2][S], s_full[2], p_full[2][4],
-    // o_final[2], o_free[2], drain[2]
-    static constexpr int kNumBars = 4 + 3 * kStages + 16;
+    // q_full[2][2], q_empty[2][2] (set, tile), ring_full[S], ring_empty[2][S], s_full[2],
+    // p_full[2][4], o_final[2], o_free[2], drain[2]
+    static constexpr int kNumBars = 8 + 3 * kStages + 16;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, 4 queue counters
     static constexpr int kFixOff = (kMiscOff + 24 + 15) & ~15;  // queue of sharp rows: kPPFixSlots x 16 B
     static constexpr int kSmemBytes = kFixOff + kPPFixSlots * 16 + 1024;  // + alignment slack
@@ -450,15 +455,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                       int64_t osb, int64_t osh, int64_t ost, float* __restrict__ lse, int BH, int H,
                       int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
                       int* status, const __grid_constant__ PPRaw raw) {
-    using C = PPCfg<D>;
+    using C = PPCfg<D, TWO>;
     constexpr int NS = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* q_full = bars;            // [2]
-    uint64_t* q_empty = bars + 2;       // [2]
-    uint64_t* ring_full = bars + 4;     // [NS]
+    uint64_t* q_full = bars;            // [2][2]: Q set s, tile x at 2s + x
+    uint64_t* q_empty = bars + 4;       // [2][2]
+    uint64_t* ring_full = bars + 8;     // [NS]
     uint64_t* ring_empty = ring_full + NS;  // [2][NS]: tile x's issuer is done with the stage
     uint64_t* s_full = ring_empty + 2 * NS;  // [2]
     uint64_t* p_full = s_full + 2;       // [2][4]: P of tile x, part s, is in TMEM
@@ -485,9 +490,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     const int n_items = single ? n_qt * BH : n_pairs;
 
     if (threadIdx.x == 0) {
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < 4; ++x) {
             ptx::mbar_init(q_full + x, 1);
             ptx::mbar_init(q_empty + x, 1);
+        }
+        for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(s_full + x, 1);
             for (int c = 0; c < 4; ++c) ptx::mbar_init(p_full + 4 * x + c, 4);  // one arrival per warp
             ptx::mbar_init(o_final + x, 1);
@@ -538,12 +545,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (!ok || (x == 1 && !it.hasB)) break;
-                    if (nq[x] > 0) ok = ptx::mbar_wait(q_empty + x, (nq[x] - 1) & 1, wait_limit_ns, abort_flag);
+                    // the n-th Q tile of side x goes to set n % kQSets, once that set's previous
+                    // tile (n - kQSets) is no longer read
+                    const int n = nq[x], qb = 2 * (n % C::kQSets) + x;
+                    if (n >= C::kQSets)
+                        ok = ptx::mbar_wait(q_empty + qb, ((n / C::kQSets) - 1) & 1, wait_limit_ns, abort_flag);
                     if (!ok) break;
-                    uint8_t* dst = smem + C::kQOff + x * C::kTileBytes;
-                    ptx::mbar_arrive_expect_tx(q_full + x, C::kTileBytes);
+                    uint8_t* dst = smem + C::kQOff + qb * C::kTileBytes;
+                    ptx::mbar_arrive_expect_tx(q_full + qb, C::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
-                        ptx::tma_load_4d(dst + c * C::kBoxBytes, &tm_q, q_full + x, c * 64, it.qt[x] * 128, it.h, it.b);
+                        ptx::tma_load_4d(dst + c * C::kBoxBytes, &tm_q, q_full + qb, c * 64, it.qt[x] * 128, it.h, it.b);
                     ++nq[x];
                 }
                 for (int kt = it.k0; kt <= it.k1 && ok; ++kt) {
@@ -691,7 +702,6 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
             const uint32_t lo_k = (uint32_t)umma::smem_desc(0, 16, 1024);              // K-major LBO field
             const uint32_t lo_v = (uint32_t)umma::smem_desc(0, C::kBoxBytes, 1024);   // MN-major LBO field
-            const uint32_t q_lo = (ptx::smem_u32(smem + C::kQOff + x * C::kTileBytes) >> 4) | lo_k;
             const uint32_t ring_lo = ptx::smem_u32(smem + C::kRingOff) >> 4;
             constexpr uint32_t kStageLo = C::kTileBytes >> 4;
             uint64_t* my_empty = ring_empty + x * NS;
@@ -710,7 +720,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const bool mine = x == 0 || it.hasB;
                 const int f = it.f[x], l = it.l[x];
                 const bool prec = pp_precise(it.qt[x], W);
-                if (mine) ok = pp_wait_warp(q_full + x, ni & 1, wait_limit_ns, abort_flag);
+                // this item's Q_x: the ni-th of side x, in set ni % kQSets
+                const int qb = 2 * (ni % C::kQSets) + x;
+                const uint32_t q_lo = (ptx::smem_u32(smem + C::kQOff + qb * C::kTileBytes) >> 4) | lo_k;
+                if (mine) ok = pp_wait_warp(q_full + qb, (ni / C::kQSets) & 1, wait_limit_ns, abort_flag);
                 if (!ok) break;
                 int pend = -1;
                 bool first_pv = true;
@@ -771,7 +784,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                             }
                             ptx::tc_commit_one(s_full + x);
                             ++ns;
-                            if (kt == l) ptx::tc_commit_one(q_empty + x);
+                            if (kt == l) ptx::tc_commit_one(q_empty + qb);
                             pend = kt;
                         }
                         release(stk, use);
@@ -957,9 +970,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     if (*abort_flag) {
         if (warp == 0 && lane == 0) {
             // let every TMA load this CTA issued land before its shared memory goes away
+            // (the last Q tile of each set: the latest use of that set's barrier)
 #pragma unroll
             for (int x = 0; x < 2; ++x)
-                if (nq[x] > 0) ptx::mbar_wait(q_full + x, (nq[x] - 1) & 1, kPPDrainLimitNs, nullptr);
+                for (int n = nq[x] - 1; n >= 0 && n >= nq[x] - C::kQSets; --n)
+                    ptx::mbar_wait(q_full + 2 * (n % C::kQSets) + x, (n / C::kQSets) & 1, kPPDrainLimitNs, nullptr);
             for (uint32_t st = 0; st < (uint32_t)NS && st < loads; ++st) {
                 const uint32_t t = st + ((loads - 1 - st) / NS) * NS;
                 ptx::mbar_wait(ring_full + st, (t / NS) & 1, kPPDrainLimitNs, nullptr);

@@ -89,7 +89,7 @@ std::map<int, DeviceState> g_dev;
 template <int D, bool LSE, bool TWO>
 cudaError_t set_pp_attrs(bool* regs_ok) {
     cudaError_t e = cudaFuncSetAttribute(swa::prefill_pp_kernel<D, LSE, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         swa::PPCfg<D>::kSmemBytes);
+                                         swa::PPCfg<D, TWO>::kSmemBytes);
     cudaFuncAttributes a;
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, swa::prefill_pp_kernel<D, LSE, TWO>);
     if (e == cudaSuccess && a.numRegs != swa::kPPLaunchRegs) *regs_ok = false;
@@ -430,13 +430,14 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
             kern<<<G, swa::kPPThreads, smem, s>>>(mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H,
                                                  (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status, raw);
         };
-        constexpr int S128 = swa::PPCfg<128>::kSmemBytes, S64 = swa::PPCfg<64>::kSmemBytes;
+        constexpr int S128 = swa::PPCfg<128, false>::kSmemBytes, S64 = swa::PPCfg<64, false>::kSmemBytes;
+        constexpr int S128t = swa::PPCfg<128, true>::kSmemBytes, S64t = swa::PPCfg<64, true>::kSmemBytes;
         if (D == 128) {
-            if (lse) two ? launch(swa::prefill_pp_kernel<128, true, true>, S128) : launch(swa::prefill_pp_kernel<128, true, false>, S128);
-            else two ? launch(swa::prefill_pp_kernel<128, false, true>, S128) : launch(swa::prefill_pp_kernel<128, false, false>, S128);
+            if (lse) two ? launch(swa::prefill_pp_kernel<128, true, true>, S128t) : launch(swa::prefill_pp_kernel<128, true, false>, S128);
+            else two ? launch(swa::prefill_pp_kernel<128, false, true>, S128t) : launch(swa::prefill_pp_kernel<128, false, false>, S128);
         } else {
-            if (lse) two ? launch(swa::prefill_pp_kernel<64, true, true>, S64) : launch(swa::prefill_pp_kernel<64, true, false>, S64);
-            else two ? launch(swa::prefill_pp_kernel<64, false, true>, S64) : launch(swa::prefill_pp_kernel<64, false, false>, S64);
+            if (lse) two ? launch(swa::prefill_pp_kernel<64, true, true>, S64t) : launch(swa::prefill_pp_kernel<64, true, false>, S64);
+            else two ? launch(swa::prefill_pp_kernel<64, false, true>, S64t) : launch(swa::prefill_pp_kernel<64, false, false>, S64);
         }
     } else {
         const int64_t nrows = B * H * T;
