@@ -592,8 +592,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             const uint64_t desc_hi = umma::smem_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
             const uint32_t lo_k = (uint32_t)umma::smem_desc(0, 16, 1024);              // K-major LBO field
             const uint32_t lo_v = (uint32_t)umma::smem_desc(0, C::kBoxBytes, 1024);   // MN-major LBO field
-            const uint32_t q_lo[2] = {(ptx::smem_u32(smem + C::kQOff) >> 4) | lo_k,
-                                      (ptx::smem_u32(smem + C::kQOff + C::kTileBytes) >> 4) | lo_k};
+            const uint32_t q_base = ptx::smem_u32(smem + C::kQOff) >> 4;
             const uint32_t ring_lo = ptx::smem_u32(smem + C::kRingOff) >> 4;
             constexpr uint32_t kStageLo = C::kTileBytes >> 4;
             uint32_t L = 0;               // K/V tiles consumed so far (same count as the producer)
@@ -606,9 +605,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 const PPItem it = pp_decode(u, BH, H, n_qt, T, W, single);
                 const int nx = it.hasB ? 2 : 1;
                 const bool prec[2] = {pp_precise(it.qt[0], W), pp_precise(it.qt[1], W)};
+                // this item's Q_x: the ni[x]-th of side x, in set ni[x] % kQSets
+                const int qb[2] = {2 * (ni[0] % C::kQSets), 2 * (ni[1] % C::kQSets) + 1};
+                const uint32_t q_lo[2] = {(q_base + qb[0] * (C::kTileBytes >> 4)) | lo_k,
+                                          (q_base + qb[1] * (C::kTileBytes >> 4)) | lo_k};
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (x < nx && ok) ok = pp_wait_warp(q_full + x, ni[x] & 1, wait_limit_ns, abort_flag);
+                    if (x < nx && ok) ok = pp_wait_warp(q_full + qb[x], (ni[x] / C::kQSets) & 1, wait_limit_ns, abort_flag);
                 }
                 if (!ok) break;
                 int pend[2] = {-1, -1};
@@ -666,7 +669,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                             }
                             ptx::tc_commit_one(s_full + x);
                             ++ns[x];
-                            if (kt == it.l[x]) ptx::tc_commit_one(q_empty + x);
+                            if (kt == it.l[x]) ptx::tc_commit_one(q_empty + qb[x]);
                             pend[x] = kt;
                         }
                     }
