@@ -414,6 +414,43 @@ int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W,
 /* ---- Diagnostics ---- */
 
 /*
+ * Prefill modes (swa_set_prefill_mode), for the bf16 tensor-core prefill with D 64 or 128
+ * (swa_forward, swa_forward_ex, swa_forward_lse, swa_forward_host, swa_mha_forward).
+ * Every mode meets the same bound on |output - exact|; they differ in how:
+ *   SWA_PREFILL_FAST: P (the softmax weights) is one bf16 value per key on every tile past
+ *     a head's first 128 rows (bands longer than 128 keys). A row in which one key ends up
+ *     above a quarter of the weight and some output reaches 1 in magnitude is recomputed
+ *     in fp32 by one warp per SM, over its whole band. Fastest on inputs where such rows
+ *     are rare (N(0,1) scores); inputs whose rows are mostly dominated by a few keys make
+ *     almost every row such a row and run 100 to 1000 times slower.
+ *   SWA_PREFILL_ADAPTIVE: a tile carries P as two bf16 parts (hi + lo, and a second P.V
+ *     product) for every warp of 32 rows in which a key could end up above a quarter of its
+ *     row's weight; no row needs recomputing. About a fifth slower than FAST on N(0,1)
+ *     inputs, and within a few times of it on any input.
+ *   SWA_PREFILL_AUTO (the default): FAST until a launch meets more than a few such rows in
+ *     one SM's work, then ADAPTIVE for every later launch on that device (see
+ *     swa_prefill_auto_state). Results are within the bound either way, but not bitwise the
+ *     same across the switch.
+ * The modes are process-wide settings read at each launch.
+ */
+#define SWA_PREFILL_AUTO 0
+#define SWA_PREFILL_ADAPTIVE 1
+#define SWA_PREFILL_FAST 2
+
+/*
+ * swa_set_prefill_mode: set the prefill mode (above) for later launches; returns the
+ * previous mode, or -1 (and sets the last error) for an unknown mode.
+ */
+int swa_set_prefill_mode(int mode);
+
+/*
+ * swa_prefill_auto_state: whether SWA_PREFILL_AUTO has switched to adaptive on the current
+ * device (1) or not (0); clear != 0 switches it back. Synchronous (a copy from or to the
+ * device). Returns -1 (and sets the last error) if the copy fails.
+ */
+int swa_prefill_auto_state(int clear);
+
+/*
  * swa_set_wait_limit_ns: time limit of every bounded wait inside the kernels, in
  * nanoseconds (default 2e9, or the SWA_WAIT_LIMIT_NS environment variable). A wait
  * that runs past it makes the kernel record SWA_ERR_TIMEOUT, let its in-flight copies

@@ -356,6 +356,26 @@ def backward_cta_tile(u, B, H, T, W, kv):
     return None if rc != 0 else (b.value, h.value, t.value)
 
 
+PREFILL_AUTO, PREFILL_ADAPTIVE, PREFILL_FAST = 0, 1, 2
+
+
+def set_prefill_mode(mode):
+    """Set the bf16 prefill mode (PREFILL_AUTO, PREFILL_ADAPTIVE or PREFILL_FAST, see
+    swa_set_prefill_mode) for later launches; returns the previous mode."""
+    prev = _native.lib().swa_set_prefill_mode(int(mode))
+    if prev < 0:
+        raise SwaError(1, _native.lib().swa_last_error().decode())
+    return prev
+
+
+def prefill_auto_state(clear=False):
+    """1 if PREFILL_AUTO has switched to adaptive on the current device, else 0; clear resets it."""
+    v = _native.lib().swa_prefill_auto_state(1 if clear else 0)
+    if v < 0:
+        raise SwaError(4, _native.lib().swa_last_error().decode())
+    return v
+
+
 def valid_slots(pos, W):
     """Number of valid ring slots (slots 0..n-1) for a stream at position pos."""
     return _native.lib().swa_decode_valid_slots(pos, W)

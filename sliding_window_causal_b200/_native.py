@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(_HERE, "_swa.so")
 EXPORTS = ("swa_forward", "swa_forward_ex", "swa_forward_host", "swa_band_weights", "swa_decode", "swa_decode_noalloc",
            "swa_chunk_forward", "swa_ring_append", "swa_mha_forward", "swa_mha_workspace_bytes",
            "swa_forward_lse", "swa_backward", "swa_backward_workspace_bytes", "swa_device_status", "swa_last_error", "swa_prefill_tile_class", "swa_prefill_work_item", "swa_backward_cta_tile", "swa_decode_valid_slots", "swa_decode_split_plan",
-           "swa_set_wait_limit_ns", "swa_timeout_probe")
+           "swa_set_wait_limit_ns", "swa_timeout_probe", "swa_set_prefill_mode", "swa_prefill_auto_state")
 
 SWA_F32, SWA_BF16 = 0, 1
 STATUS_NAMES = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED",
@@ -78,6 +78,10 @@ def lib(path=None):
     h.swa_prefill_work_item.restype = i32
     h.swa_backward_cta_tile.argtypes = [i64] * 5 + [i32] + [pi64] * 3
     h.swa_backward_cta_tile.restype = i32
+    h.swa_set_prefill_mode.argtypes = [i32]
+    h.swa_set_prefill_mode.restype = i32
+    h.swa_prefill_auto_state.argtypes = [i32]
+    h.swa_prefill_auto_state.restype = i32
     h.swa_decode_valid_slots.argtypes = [i64, i64]
     h.swa_decode_valid_slots.restype = i64
     h.swa_decode_split_plan.argtypes = [i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int32),

@@ -89,6 +89,16 @@ static_assert(kPPParts == 1 || kPPParts == 2 || kPPParts == 4, "parts of a tile'
 // the output almost undamped, on top of the output's own bf16 rounding (2^-8 relative).
 constexpr float kPPSharpShare = 0.25f;
 constexpr float kPPSharpOut = 1.0f;
+// ADAPT (a kernel template argument): a softmax warp writes hi + lo parts of P on any tile
+// where one of its rows meets a key that could end up above a quarter of the row's weight,
+// and the MMA issuer adds the second P.V product for those warps' rows, so that no row
+// becomes sharp. On N(0,1) inputs this costs about a fifth of the throughput; on inputs
+// whose rows are dominated by a few keys it saves recomputing nearly every row. Without
+// ADAPT, once one CTA has recomputed kPPAdaptAfter sharp rows the kernel sets *auto_flag
+// (when given: a word of host memory mapped for the device), which the host reads to run
+// later launches with ADAPT.
+constexpr int kPPAdaptAfter = 8;
+
 // Sharp rows go through a queue in shared memory to warp 2 (otherwise idle), which
 // recomputes them while the softmax warps carry on; a full queue makes a softmax thread
 // wait for a free slot.
@@ -121,7 +131,8 @@ struct PPCfg {
     // p_full[2][4], o_final[2], o_free[2], drain[2]
     static constexpr int kNumBars = 8 + 3 * kStages + 16;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, 4 queue counters
-    static constexpr int kFixOff = (kMiscOff + 24 + 15) & ~15;  // queue of sharp rows: kPPFixSlots x 16 B
+    static constexpr int kLoOff = (kMiscOff + 24 + 15) & ~15;  // low-part flags [2 tiles][2 parities][4 warps]
+    static constexpr int kFixOff = kLoOff + 64;                 // queue of sharp rows: kPPFixSlots x 16 B
     static constexpr int kSmemBytes = kFixOff + kPPFixSlots * 16 + 1024;  // + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     __device__ static constexpr uint32_t colS(int x) { return 128u * x; }
@@ -180,6 +191,20 @@ __device__ __forceinline__ bool pp_wait_warp(uint64_t* bar, uint32_t parity, uin
 
 __device__ __forceinline__ bool pp_precise(int qt, int W) { return qt == 0 || W <= kPPPreciseWindow; }
 
+// Which warps of tile x's softmax wrote low parts of P for the side-x tile number t (the
+// flags of its parity; read after the tile's first part was handed over): dis[w] disables
+// the 32 TMEM lanes of warp w in the second P.V product when it did not. Returns whether
+// any did.
+__device__ __forceinline__ bool pp_lo_lanes(volatile const uint32_t* lo_flag, int x, uint32_t t, uint32_t (&dis)[4]) {
+    uint32_t w[4];  // one 16-byte load (the four flags of a tile are 16-byte aligned)
+    asm volatile("ld.volatile.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "r"(ptx::smem_u32(const_cast<const uint32_t*>(lo_flag + 4 * (2 * x + (t & 1))))));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dis[j] = w[j] != 0u ? 0u : 0xFFFFFFFFu;
+    return (w[0] | w[1] | w[2] | w[3]) != 0u;
+}
+
 // Column of TMEM (relative to the S buffer) that holds P for keys 16kk..16kk+15: keys
 // 32c..32c+31 are packed into columns 32c..32c+15 (and, for precise tiles, the low parts
 // into 32c+16..32c+31), so that P only ever overwrites S values already read.
@@ -222,6 +247,46 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
     ptx::tmem_st_wait();
 }
 
+// P = exp2(s*c - mu) for the thread's 128 scores v (c = scale_log2), written over S as bf16
+// in columns 32c..32c+15 of each 32-column chunk; LO = 1 also writes the low parts
+// P - bf16(P), rounded to bf16, in columns 32c+16..32c+31, LO = 0 nothing. after_part(s) runs once part s's stores are issued and the next chunk's
+// arithmetic is done. Returns the sum of the weights as written (hi + lo).
+template <int LO, typename AfterPart>
+__device__ __forceinline__ float pp_exps(uint32_t scol, const uint32_t (&v)[4][32], float scale_log2, float mu,
+                                         AfterPart after_part) {
+    const ptx::f32x2 sc = {scale_log2, scale_log2}, nm = {-mu, -mu};
+    ptx::f32x2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const ptx::f32x2 s2 = {__uint_as_float(v[c][2 * t]), __uint_as_float(v[c][2 * t + 1])};
+            const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
+            const float e0 = ptx::ex2(z.x), e1 = ptx::ex2(z.y);
+            ph[t] = ptx::pack_bf16x2(e0, e1);
+            if (LO == 1) {
+                const ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
+                pl[t] = ptx::pack_bf16x2(e0 - w.x, e1 - w.y);
+                acc[(t + 2) & 3] = ptx::add2(acc[(t + 2) & 3], {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
+                acc[t & 3] = ptx::add2(acc[t & 3], w);
+            } else {
+                acc[t & 3] = ptx::add_bf16x2_f32(ph[t], acc[t & 3]);
+            }
+        }
+        // the previous part's stores have had this chunk's arithmetic to land
+        if (c > 0 && c % (4 / kPPParts) == 0) after_part(c / (4 / kPPParts) - 1);
+        ptx::tmem_st16(scol + 32 * c, ph);
+        if (LO == 1) ptx::tmem_st16(scol + 32 * c + 16, pl);
+    }
+    after_part(kPPParts - 1);
+    return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+}
+
+struct PPNoPublish {
+    __device__ void operator()(bool) const {}
+};
+
 // One tile of one row: the thread's 128 scores are read from TMEM in one round trip,
 // masked on edge tiles, reduced to the row maximum (log2 units), and P = exp2(s*c - m)
 // is written back over the S columns as bf16 pairs (round to nearest): keys 32c..32c+31
@@ -237,16 +302,22 @@ __device__ __forceinline__ void pp_rescale(uint32_t ocol, uint32_t scol, int chu
 // is rescaled, for callers whose last P.V product may still be in flight. after_part(s)
 // runs (warp-uniformly) once the stores of part s of P (keys 128s/kPPParts ..) have been
 // issued and the next chunk's arithmetic is done, so that the caller can hand that part
-// to the MMA issuer while the rest of the tile is computed.
-// Returns the row's largest scaled score in the tile (log2 units; -inf if none is in band).
+// to the MMA issuer while the rest of the tile is computed. ADAPT (with PRECISE false): the
+// warp chooses hi + lo parts for this tile when one of its rows meets a key that could end
+// up above a quarter of the row's weight, or always when force is set; publish(bool) tells
+// the caller which.
+// Returns the row's largest scaled score in the tile (log2 units; -inf if none is in band,
+// or if the tile's weights were written in two parts).
 struct PPNoPart {
     __device__ void operator()(int) const {}
 };
 
-template <int D, int MASK, bool PRECISE, typename BeforeRescale, typename AfterPart = PPNoPart>
+template <int D, int MASK, bool PRECISE, bool ADAPT = false, typename BeforeRescale, typename AfterPart = PPNoPart,
+          typename Publish = PPNoPublish>
 __device__ __forceinline__ float pp_tile(uint32_t scol, uint32_t ocol, float scale_log2, float& m,
                                         float& l, int cmin, int cmax, int cmin2, int cmax2,
-                                        BeforeRescale before_rescale, AfterPart after_part = AfterPart()) {
+                                        BeforeRescale before_rescale, AfterPart after_part = AfterPart(),
+                                        Publish publish = Publish(), bool force = false) {
     uint32_t v[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) ptx::tmem_ld32(scol + 32 * c, v[c]);
@@ -299,33 +370,24 @@ __device__ __forceinline__ float pp_tile(uint32_t scol, uint32_t ocol, float sca
     }
     if (m == -INFINITY) m = tm;  // first in-band keys of the row (or still none)
     const float mu = m == -INFINITY ? 0.f : m;
-    const ptx::f32x2 sc = {scale_log2, scale_log2}, nm = {-mu, -mu};
-    ptx::f32x2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t ph[16], pl[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const ptx::f32x2 s2 = {__uint_as_float(v[c][2 * t]), __uint_as_float(v[c][2 * t + 1])};
-            const ptx::f32x2 z = ptx::fma2(s2, sc, nm);
-            const float e0 = ptx::ex2(z.x), e1 = ptx::ex2(z.y);
-            ph[t] = ptx::pack_bf16x2(e0, e1);
-            if (PRECISE) {
-                const ptx::f32x2 w = {ptx::bf16lo_f32(ph[t]), ptx::bf16hi_f32(ph[t])};
-                pl[t] = ptx::pack_bf16x2(e0 - w.x, e1 - w.y);
-                acc[(t + 2) & 3] = ptx::add2(acc[(t + 2) & 3], {ptx::bf16lo_f32(pl[t]), ptx::bf16hi_f32(pl[t])});
-                acc[t & 3] = ptx::add2(acc[t & 3], w);
-            } else {
-                acc[t & 3] = ptx::add_bf16x2_f32(ph[t], acc[t & 3]);
-            }
+    if (ADAPT) {
+        // A key of this tile can end up above a quarter of its row's weight (the test for a
+        // sharp row) only if its weight exceeds a third of the weight met before the tile:
+        // w > (l + w)/4 needs 3w > l, and later tiles only add weight. Such a row, or any in
+        // the warp, takes P as hi + lo parts; the warp tells the MMA issuer (publish) before
+        // it hands the first part over, and the issuer's second P.V product leaves the
+        // rows of the other warps unchanged.
+        const bool flag = force || (tm != -INFINITY && 3.f * ptx::ex2(tm - mu) > l);
+        const bool any = __any_sync(0xffffffffu, flag);
+        publish(any);
+        if (any) {
+            l += pp_exps<1>(scol, v, scale_log2, mu, after_part);
+            return -INFINITY;  // every weight of the tile is carried in two parts
         }
-        // the previous part's stores have had this chunk's arithmetic to land
-        if (c > 0 && c % (4 / kPPParts) == 0) after_part(c / (4 / kPPParts) - 1);
-        ptx::tmem_st16(scol + 32 * c, ph);
-        if (PRECISE) ptx::tmem_st16(scol + 32 * c + 16, pl);
+        l += pp_exps<0>(scol, v, scale_log2, mu, after_part);
+        return tm;
     }
-    after_part(kPPParts - 1);
-    l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+    l += pp_exps<PRECISE ? 1 : 0>(scol, v, scale_log2, mu, after_part);
     return tm;
 }
 
@@ -452,14 +514,15 @@ __device__ __forceinline__ bool pp_push_sharp(uint32_t* fix_head, const uint32_t
 }
 
 // LSE: also write the natural log-sum-exp of each row (a separate instantiation, so that
-// the plain prefill keeps its register allocation).
-template <int D, bool LSE = false, bool TWO = false>
+// the plain prefill keeps its register allocation). ADAPT: hi + lo P chosen per warp and
+// tile (above); likewise its own instantiation, so that the kernel without it is not slowed.
+template <int D, bool LSE = false, bool TWO = false, bool ADAPT = false>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                       int64_t osb, int64_t osh, int64_t ost, float* __restrict__ lse, int BH, int H,
                       int T, int W, int n_qt, float scale_log2, uint64_t wait_limit_ns,
-                      int* status, const __grid_constant__ PPRaw raw) {
+                      int* status, const __grid_constant__ PPRaw raw, int* auto_flag) {
     using C = PPCfg<D, TWO>;
     constexpr int NS = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -485,6 +548,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     uint32_t* fix_beat = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 16);
     uint32_t* fix_tail = reinterpret_cast<uint32_t*>(smem + C::kMiscOff + 20);
     uint4* fix_slot = reinterpret_cast<uint4*>(smem + C::kFixOff);
+    // lo_flag[4 * (2x + parity) + w]: warp w of tile x's softmax wrote low parts of P for the
+    // x-tile of that parity (counted in tiles of side x); read by the MMA issuer once the
+    // tile's first part is handed over
+    volatile uint32_t* lo_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kLoOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, g = blockIdx.x;
@@ -518,6 +585,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         *fix_beat = 0;
         *fix_tail = 0;
         for (int q = 0; q < kPPFixSlots; ++q) fix_slot[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 16; ++q) lo_flag[q] = 0u;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -533,6 +601,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    constexpr bool adapt = ADAPT;
 
     uint32_t loads = 0;  // producer: K/V tiles issued so far
     int nq[2] = {0, 0};  // producer: Q tiles issued per side
@@ -639,18 +708,28 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                             // must be free if it starts the item
                             if (first_pv[x] && ni[x] > 0)
                                 ok = pp_wait_warp(o_free + x, (ni[x] - 1) & 1, wait_limit_ns, abort_flag);
+                            // low parts: every lane on tiles that always carry them, else the lanes
+                            // of the softmax warps that wrote them for this tile
+                            bool lo_parts = prec[x];
+                            uint32_t dis[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                             for (int part = 0; part < kPPParts && ok; ++part) {
                                 ok = pp_wait_warp(p_full + 4 * x + part, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
                                 if (!ok) break;
                                 ptx::tc_fence_after();
+                                if (part == 0 && adapt && !prec[x]) lo_parts = pp_lo_lanes(lo_flag, x, ns[x] - 1, dis);
                                 constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
 #pragma unroll
                                 for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                     ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
                                                     desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
                                                     (!first_pv[x] || kk > 0) ? 1u : 0u);
-                                if (prec[x]) {
+                                if (lo_parts && adapt) {
+#pragma unroll
+                                    for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                        ptx::mma_ts_one_masked(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                               desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u, dis);
+                                } else if (lo_parts) {
 #pragma unroll
                                     for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                         ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
@@ -749,18 +828,28 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                             if (first_pv && ni > 0)
                                 ok = pp_wait_warp(o_free + x, (ni - 1) & 1, wait_limit_ns, abort_flag);
                             const uint32_t v_lo = (ring_lo + stv * kStageLo) | lo_v;
+                            // low parts: every lane on tiles that always carry them, else the lanes
+                            // of the softmax warps that wrote them for this tile
+                            bool lo_parts = prec;
+                            uint32_t dis[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                             for (int part = 0; part < kPPParts && ok; ++part) {
                                 ok = pp_wait_warp(p_full + 4 * x + part, (ns - 1) & 1, wait_limit_ns, abort_flag);
                                 if (!ok) break;
                                 ptx::tc_fence_after();
+                                if (part == 0 && adapt && !prec) lo_parts = pp_lo_lanes(lo_flag, x, ns - 1, dis);
                                 constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
 #pragma unroll
                                 for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                     ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
                                                     desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
                                                     (!first_pv || kk > 0) ? 1u : 0u);
-                                if (prec) {
+                                if (lo_parts && adapt) {
+#pragma unroll
+                                    for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
+                                        ptx::mma_ts_one_masked(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
+                                                               desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o, 1u, dis);
+                                } else if (lo_parts) {
 #pragma unroll
                                     for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                         ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
@@ -844,6 +933,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             const int fb = (int)ent.x, fh = (int)ent.y, fi = (int)ent.z;
             pp_fix_row<D>(raw, fb, fh, fi, W, scale_log2, out + fb * osb + fh * osh + (int64_t)fi * ost,
                           LSE ? lse + ((int64_t)fb * H + fh) * T + fi : nullptr, lane);
+            // inputs that make this many rows sharp in one CTA run adaptive from the next launch
+            if (!ADAPT && auto_flag != nullptr && sl + 1 == (uint32_t)kPPAdaptAfter && lane == 0) {
+                *reinterpret_cast<volatile int*>(auto_flag) = 1;
+                __threadfence_system();
+            }
             __syncwarp();
             if (lane == 0) *reinterpret_cast<volatile uint32_t*>(fix_tail) = sl + 1;  // slot free again
         }
@@ -890,7 +984,20 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(p_full + 4 * x + part);
                 };
-                if (edge) {
+                // whether this warp wrote low parts of P, for the MMA issuer (before part 0's
+                // arrival, which releases it)
+                const auto publish = [&](bool lo_parts) {
+                    if (lane == 0) lo_flag[4 * (2 * x + ((ns - 1) & 1)) + (warp & 3)] = lo_parts ? 1u : 0u;
+                };
+                if (adapt) {
+                    // (tiles that always carry low parts take the same code with force set)
+                    if (edge)
+                        t_np = fmaxf(t_np, pp_tile<D, 1, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0,
+                                                                      -1, none, hand, publish, precise));
+                    else
+                        t_np = fmaxf(t_np, pp_tile<D, 0, false, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0,
+                                                                      -1, none, hand, publish, precise));
+                } else if (edge) {
                     if (precise) pp_tile<D, 1, true>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand);
                     else t_np = fmaxf(t_np, pp_tile<D, 1, false>(scol, ocol, scale_log2, m_ref, l, cmin, cmax, 0, -1, none, hand));
                 } else {

@@ -190,6 +190,17 @@ __device__ __forceinline__ void mma_ts_one(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
+// mma_ts_one that leaves some lanes of D unchanged: bit j of dis[w] set keeps TMEM lane
+// 32w + j (row 32w + j of the product) as it is.
+__device__ __forceinline__ void mma_ts_one_masked(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate, const uint32_t (&dis)[4]) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(dis[0]), "r"(dis[1]), "r"(dis[2]), "r"(dis[3])
+        : "memory");
+}
+
 #define SWA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
                   "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
 #define SWA_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <type_traits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -53,6 +54,7 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<uint64_t> g_wait_limit{0};
+std::atomic<int> g_prefill_mode{SWA_PREFILL_AUTO};
 
 uint64_t env_wait_limit() {
     static uint64_t v = [] {
@@ -80,20 +82,30 @@ struct DeviceState {
     int* status = nullptr;  // device address of g_swa_status
     int num_sms = 0;
     bool pp_regs_ok = false;  // the persistent prefill kernels use exactly kPPLaunchRegs
+    // SWA_PREFILL_AUTO's switch: a word of pinned host memory that the prefill kernel without
+    // adaptive P sets (through its device mapping) when its inputs make many rows sharp
+    volatile int* auto_host = nullptr;
+    int* auto_dev = nullptr;
 };
 std::map<int, DeviceState> g_dev;
 
-// The eight tensor-core prefill kernels (D 64/128, with and without the log-sum-exp, one or
-// two MMA issuers): set the shared-memory size, and check that each was compiled with the
-// kPPLaunchRegs registers per thread that its register split assumes.
-template <int D, bool LSE, bool TWO>
-cudaError_t set_pp_attrs(bool* regs_ok) {
-    cudaError_t e = cudaFuncSetAttribute(swa::prefill_pp_kernel<D, LSE, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         swa::PPCfg<D, TWO>::kSmemBytes);
+// The sixteen tensor-core prefill kernels (D 64/128, with and without the log-sum-exp, one or
+// two MMA issuers, with and without adaptive P): set the shared-memory size, and check that
+// each was compiled with the kPPLaunchRegs registers per thread that its register split
+// assumes.
+template <int D, bool LSE, bool TWO, bool ADAPT>
+cudaError_t set_pp_attrs_one(bool* regs_ok) {
+    cudaError_t e = cudaFuncSetAttribute(swa::prefill_pp_kernel<D, LSE, TWO, ADAPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, swa::PPCfg<D, TWO>::kSmemBytes);
     cudaFuncAttributes a;
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, swa::prefill_pp_kernel<D, LSE, TWO>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, swa::prefill_pp_kernel<D, LSE, TWO, ADAPT>);
     if (e == cudaSuccess && a.numRegs != swa::kPPLaunchRegs) *regs_ok = false;
     return e;
+}
+template <int D, bool LSE, bool TWO>
+cudaError_t set_pp_attrs(bool* regs_ok) {
+    cudaError_t e = set_pp_attrs_one<D, LSE, TWO, false>(regs_ok);
+    return e == cudaSuccess ? set_pp_attrs_one<D, LSE, TWO, true>(regs_ok) : e;
 }
 
 template <int D>
@@ -127,6 +139,19 @@ int device_state(DeviceState** out) {
             st.status = nullptr;
             return cuda_fail(e, "cudaGetSymbolAddress(status)");
         }
+    }
+    if (!st.auto_dev) {
+        int* h = nullptr;
+        e = cudaHostAlloc(reinterpret_cast<void**>(&h), sizeof(int), cudaHostAllocMapped);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaHostAlloc(prefill mode word)");
+        *h = 0;
+        e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&st.auto_dev), h, 0);
+        if (e != cudaSuccess) {
+            cudaFreeHost(h);
+            st.auto_dev = nullptr;
+            return cuda_fail(e, "cudaHostGetDevicePointer(prefill mode word)");
+        }
+        st.auto_host = h;
     }
     if (!st.attrs_set) {
         e = cudaSuccess;
@@ -426,19 +451,30 @@ int forward_impl(const char* fn, const void* q, const void* k, const void* v, vo
         // waiting on the other's P. Longer bands keep the single issuer, whose ping-pong order
         // completes each tile's scores sooner.
         const bool two = Wi <= swa::kPPTwoIssuerWindow;
+        // adaptive P when asked for, or when an earlier launch on this device in AUTO mode
+        // met inputs that make many rows sharp (the kernel without it sets the word)
+        const int mode = g_prefill_mode.load();
+        const bool adapt = mode == SWA_PREFILL_ADAPTIVE || (mode == SWA_PREFILL_AUTO && *ds->auto_host != 0);
+        int* auto_flag = mode == SWA_PREFILL_AUTO ? ds->auto_dev : nullptr;
         auto launch = [&](auto kern, int smem) {
             kern<<<G, swa::kPPThreads, smem, s>>>(mq, mk, mv, ob, st[3][0], st[3][1], st[3][2], lse, (int)BH, (int)H,
-                                                 (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status, raw);
+                                                 (int)T, Wi, n_qt, scale_log2, wait_limit(), ds->status, raw, auto_flag);
         };
         constexpr int S128 = swa::PPCfg<128, false>::kSmemBytes, S64 = swa::PPCfg<64, false>::kSmemBytes;
         constexpr int S128t = swa::PPCfg<128, true>::kSmemBytes, S64t = swa::PPCfg<64, true>::kSmemBytes;
-        if (D == 128) {
-            if (lse) two ? launch(swa::prefill_pp_kernel<128, true, true>, S128t) : launch(swa::prefill_pp_kernel<128, true, false>, S128);
-            else two ? launch(swa::prefill_pp_kernel<128, false, true>, S128t) : launch(swa::prefill_pp_kernel<128, false, false>, S128);
-        } else {
-            if (lse) two ? launch(swa::prefill_pp_kernel<64, true, true>, S64t) : launch(swa::prefill_pp_kernel<64, true, false>, S64);
-            else two ? launch(swa::prefill_pp_kernel<64, false, true>, S64t) : launch(swa::prefill_pp_kernel<64, false, false>, S64);
-        }
+        // one launch of the instantiation <D, lse, two, adapt>
+        auto pick = [&](auto d_tag, int smem1, int smem2) {
+            constexpr int DD = decltype(d_tag)::value;
+            if (lse) {
+                if (two) adapt ? launch(swa::prefill_pp_kernel<DD, true, true, true>, smem2) : launch(swa::prefill_pp_kernel<DD, true, true, false>, smem2);
+                else adapt ? launch(swa::prefill_pp_kernel<DD, true, false, true>, smem1) : launch(swa::prefill_pp_kernel<DD, true, false, false>, smem1);
+            } else {
+                if (two) adapt ? launch(swa::prefill_pp_kernel<DD, false, true, true>, smem2) : launch(swa::prefill_pp_kernel<DD, false, true, false>, smem2);
+                else adapt ? launch(swa::prefill_pp_kernel<DD, false, false, true>, smem1) : launch(swa::prefill_pp_kernel<DD, false, false, false>, smem1);
+            }
+        };
+        if (D == 128) pick(std::integral_constant<int, 128>(), S128, S128t);
+        else pick(std::integral_constant<int, 64>(), S64, S64t);
     } else {
         const int64_t nrows = B * H * T;
         const int64_t blocks = (nrows + swa::kSimtWarps - 1) / swa::kSimtWarps;
@@ -501,6 +537,22 @@ uint64_t swa_set_wait_limit_ns(uint64_t ns) {
     uint64_t prev = wait_limit();
     g_wait_limit.store(ns);
     return prev;
+}
+
+int swa_set_prefill_mode(int mode) {
+    if (mode != SWA_PREFILL_AUTO && mode != SWA_PREFILL_ADAPTIVE && mode != SWA_PREFILL_FAST) {
+        fail(SWA_ERR_INVALID_ARG, "swa_set_prefill_mode: mode %d", mode);
+        return -1;
+    }
+    return g_prefill_mode.exchange(mode);
+}
+
+int swa_prefill_auto_state(int clear) {
+    DeviceState* ds;
+    if (device_state(&ds)) return -1;
+    const int v = *ds->auto_host;
+    if (clear) *ds->auto_host = 0;
+    return v;
 }
 
 int swa_prefill_tile_class(int64_t T, int64_t W, int64_t bm, int64_t bn, int64_t qt, int64_t kt) {

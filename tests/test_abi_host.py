@@ -276,3 +276,18 @@ def test_ctypes_signatures_match_the_header():
         want = [_c_kind(t) for t in params]
         assert got == want, f"{name}: binding {got} vs header {want}"
         assert _kind(f.restype) == _c_kind(ret), f"{name}: return {f.restype} vs {ret}"
+
+
+def test_prefill_mode_setting():
+    """swa_set_prefill_mode returns the previous mode and refuses unknown ones (host only)."""
+    prev = swa.set_prefill_mode(swa.PREFILL_FAST)
+    try:
+        assert swa.set_prefill_mode(swa.PREFILL_ADAPTIVE) == swa.PREFILL_FAST
+        assert swa.set_prefill_mode(swa.PREFILL_AUTO) == swa.PREFILL_ADAPTIVE
+        with pytest.raises(swa.SwaError):
+            swa.set_prefill_mode(3)
+        with pytest.raises(swa.SwaError):
+            swa.set_prefill_mode(-1)
+        assert swa.set_prefill_mode(swa.PREFILL_AUTO) == swa.PREFILL_AUTO
+    finally:
+        swa.set_prefill_mode(prev)

@@ -9,7 +9,7 @@ import oracle
 import sliding_window_causal_b200 as swa
 from sliding_window_causal_b200 import _native, inputs
 from golden import read_moving_average
-from gpu_util import TOL, f64, max_err
+from gpu_util import TOL, f64, max_err, sharp_inputs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -248,3 +248,65 @@ def test_growing_scores_move_the_reference(D, W):
     out = run(q, k, v, W)
     ref = oracle.forward(f64(q), f64(k), f64(v), W)
     assert max_err(out, ref) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("kind", ["growing", "falling", "spikes"])
+@pytest.mark.parametrize("D,W", [(128, 4096), (64, 300), (128, 600)])
+def test_adaptive_mode_on_rows_a_few_keys_dominate(kind, D, W):
+    """Adaptive P (hi + lo parts on the tiles where a key of one of a warp's rows could end
+    up above a quarter of its row's weight, and a second P.V product for those warps'
+    rows): the inputs that make the fast mode recompute nearly every row match the oracle
+    without recomputing any, in the plain and the training forward."""
+    B, H, T = 1, 3, 1300
+    q, k, v = sharp_inputs(B, H, T, D, 50 + W + D, kind)
+    prev = swa.set_prefill_mode(swa.PREFILL_ADAPTIVE)
+    try:
+        out = run(q, k, v, W)
+        out2, _ = swa.forward_lse(q.to(DEV), k.to(DEV), v.to(DEV), W)
+        swa.device_status()
+    finally:
+        swa.set_prefill_mode(prev)
+    ref = oracle.forward(f64(q), f64(k), f64(v), W)
+    assert max_err(out, ref) <= TOL[torch.bfloat16]
+    assert max_err(out2, ref) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("B,H,T,D,W", [(1, 2, 3000, 128, 1500), (2, 2, 1000, 128, 300), (1, 3, 777, 64, 200)])
+def test_adaptive_mode_parity(B, H, T, D, W):
+    """Adaptive P on N(0,1) inputs: one and two MMA issuers, D 64 and 128, ragged T."""
+    prev = swa.set_prefill_mode(swa.PREFILL_ADAPTIVE)
+    try:
+        full_parity(B, H, T, D, W, torch.bfloat16, 11 + T + W)
+    finally:
+        swa.set_prefill_mode(prev)
+
+
+def test_auto_mode_switches_after_many_sharp_rows():
+    """In the default mode a launch whose inputs make many rows sharp (here the oldest key
+    of every band dominates) is computed with single-bf16 P and those rows recomputed; it
+    switches the device to adaptive P for later launches, which still match the oracle."""
+    prev = swa.set_prefill_mode(swa.PREFILL_AUTO)
+    try:
+        assert swa.prefill_auto_state() == 0
+        full_parity(1, 2, 1000, 128, 700, torch.bfloat16, 5)
+        assert swa.prefill_auto_state() == 0, "N(0,1) inputs make almost no row sharp"
+        q, k, v = sharp_inputs(1, 3, 1300, 128, 7, "falling")
+        out = run(q, k, v, 600)
+        assert max_err(out, oracle.forward(f64(q), f64(k), f64(v), 600)) <= TOL[torch.bfloat16]
+        assert swa.prefill_auto_state() == 1
+        full_parity(1, 2, 1000, 128, 700, torch.bfloat16, 6)
+        assert swa.prefill_auto_state(clear=True) == 1
+        assert swa.prefill_auto_state() == 0
+    finally:
+        swa.set_prefill_mode(prev)
+
+
+def test_fast_mode_never_switches():
+    prev = swa.set_prefill_mode(swa.PREFILL_FAST)
+    try:
+        q, k, v = sharp_inputs(1, 3, 1300, 128, 7, "falling")
+        out = run(q, k, v, 600)
+        assert max_err(out, oracle.forward(f64(q), f64(k), f64(v), 600)) <= TOL[torch.bfloat16]
+        assert swa.prefill_auto_state() == 0
+    finally:
+        swa.set_prefill_mode(prev)
