@@ -61,9 +61,9 @@ def _scaled(kind, captured):
 
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
-    "prefill": {"bytes": 540.9e6 + 114.7e6, "sources": "9ece501b7b5b1e12"},
-    "decode": {"bytes": _scaled("decode", 951.0e6 + 6.3e6), "sources": "be9af298ce410eec"},
-    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 17.2e6), "sources": "b3aab250fabf2a87"},
+    "prefill": {"bytes": 549.5e6 + 113.8e6, "sources": "dcf0d55e072af1d5"},
+    "decode": {"bytes": _scaled("decode", 951.0e6 + 3.7e6), "sources": "5d66f52c4894035b"},
+    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 17.2e6), "sources": "7fe0be30a01cfb5d"},
 }
 
 
