@@ -425,7 +425,7 @@ int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W,
  *     almost every row such a row and run 100 to 1000 times slower.
  *   SWA_PREFILL_ADAPTIVE: a tile carries P as two bf16 parts (hi + lo, and a second P.V
  *     product) for every warp of 32 rows in which a key could end up above a quarter of its
- *     row's weight; no row needs recomputing. About a fifth slower than FAST on N(0,1)
+ *     row's weight; no row needs recomputing. About an eighth slower than FAST on N(0,1)
  *     inputs, and within a few times of it on any input.
  *   SWA_PREFILL_AUTO (the default): FAST until a launch meets more than a few such rows in
  *     one SM's work, then ADAPTIVE for every later launch on that device (see

@@ -92,7 +92,7 @@ constexpr float kPPSharpOut = 1.0f;
 // ADAPT (a kernel template argument): a softmax warp writes hi + lo parts of P on any tile
 // where one of its rows meets a key that could end up above a quarter of the row's weight,
 // and the MMA issuer adds the second P.V product for those warps' rows, so that no row
-// becomes sharp. On N(0,1) inputs this costs about a fifth of the throughput; on inputs
+// becomes sharp. On N(0,1) inputs this costs about an eighth of the throughput; on inputs
 // whose rows are dominated by a few keys it saves recomputing nearly every row. Without
 // ADAPT, once one CTA has recomputed kPPAdaptAfter sharp rows the kernel sets *auto_flag
 // (when given: a word of host memory mapped for the device), which the host reads to run
@@ -717,14 +717,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                                 ok = pp_wait_warp(p_full + 4 * x + part, (ns[x] - 1) & 1, wait_limit_ns, abort_flag);
                                 if (!ok) break;
                                 ptx::tc_fence_after();
-                                if (part == 0 && adapt && !prec[x]) lo_parts = pp_lo_lanes(lo_flag, x, ns[x] - 1, dis);
                                 constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
 #pragma unroll
                                 for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                     ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
                                                     desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
                                                     (!first_pv[x] || kk > 0) ? 1u : 0u);
-                                if (lo_parts && adapt) {
+                                // the warps' choices, read while the tensor pipe takes the part's
+                                // products; every warp's rows: the unmasked form
+                                if (part == 0 && adapt && !prec[x]) lo_parts = pp_lo_lanes(lo_flag, x, ns[x] - 1, dis);
+                                if (lo_parts && adapt && (dis[0] | dis[1] | dis[2] | dis[3]) != 0u) {
 #pragma unroll
                                     for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                         ptx::mma_ts_one_masked(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
@@ -837,14 +839,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                                 ok = pp_wait_warp(p_full + 4 * x + part, (ns - 1) & 1, wait_limit_ns, abort_flag);
                                 if (!ok) break;
                                 ptx::tc_fence_after();
-                                if (part == 0 && adapt && !prec) lo_parts = pp_lo_lanes(lo_flag, x, ns - 1, dis);
                                 constexpr int kPer = 8 / kPPParts;  // 16-key MMA steps per part
 #pragma unroll
                                 for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                     ptx::mma_ts_one(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk),
                                                     desc_hi | (v_lo + kk * (2048 >> 4)), idesc_o,
                                                     (!first_pv || kk > 0) ? 1u : 0u);
-                                if (lo_parts && adapt) {
+                                // the warps' choices, read while the tensor pipe takes the part's
+                                // products; every warp's rows: the unmasked form
+                                if (part == 0 && adapt && !prec) lo_parts = pp_lo_lanes(lo_flag, x, ns - 1, dis);
+                                if (lo_parts && adapt && (dis[0] | dis[1] | dis[2] | dis[3]) != 0u) {
 #pragma unroll
                                     for (int kk = part * kPer; kk < (part + 1) * kPer; ++kk)
                                         ptx::mma_ts_one_masked(tmem + C::colO(x), tmem + C::colS(x) + pp_pcol(kk) + 16,
