@@ -61,9 +61,9 @@ def _scaled(kind, captured):
 
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
-    "prefill": {"bytes": 549.5e6 + 113.8e6, "sources": "dcf0d55e072af1d5"},
+    "prefill": {"bytes": 528.1e6 + 112.6e6, "sources": "fd3530d0547e2235"},
     "decode": {"bytes": _scaled("decode", 951.0e6 + 3.7e6), "sources": "5d66f52c4894035b"},
-    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 17.2e6), "sources": "7fe0be30a01cfb5d"},
+    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 16.7e6), "sources": "c0c73eb814bb0518"},
 }
 
 
