@@ -61,9 +61,9 @@ def _scaled(kind, captured):
 
 MEASURED_TRAFFIC = {
     # Mistral-shaped workload, captured at full size (prefill only on the device)
-    "prefill": {"bytes": 528.1e6 + 112.6e6, "sources": "fd3530d0547e2235"},
+    "prefill": {"bytes": 548.4e6 + 116.5e6, "sources": "c826ea2319336f9b"},
     "decode": {"bytes": _scaled("decode", 951.0e6 + 3.7e6), "sources": "5d66f52c4894035b"},
-    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 16.7e6), "sources": "c0c73eb814bb0518"},
+    "chunk": {"bytes": _scaled("chunk", 1105.4e6 + 17.4e6), "sources": "11efae5968553e54"},
 }
 
 

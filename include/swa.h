@@ -418,7 +418,7 @@ int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W,
  * (swa_forward, swa_forward_ex, swa_forward_lse, swa_forward_host, swa_mha_forward).
  * Every mode meets the same bound on |output - exact|; they differ in how:
  *   SWA_PREFILL_FAST: P (the softmax weights) is one bf16 value per key on every tile past
- *     a head's first 128 rows (bands longer than 128 keys). A row in which one key ends up
+ *     a head's first 128 rows (bands longer than 144 keys). A row in which one key ends up
  *     above a quarter of the weight and some output reaches 1 in magnitude is recomputed
  *     in fp32 by one warp per SM, over its whole band. Fastest on inputs where such rows
  *     are rare (N(0,1) scores); inputs whose rows are mostly dominated by a few keys make

@@ -71,11 +71,12 @@ constexpr float kPPRescaleThreshold = 8.0f;  // lazy O rescale: the max may grow
 // couple of weights decide each output and |out| can exceed 2, so a single bf16 P would
 // use up the error budget left by the output's own bf16 rounding. With single-bf16 P, such
 // rows are found sharp at the epilogue and recomputed one by one on the CUDA cores; for
-// bands of up to 128 keys and N(0,1) scores so many rows are sharp that the one
+// bands of up to 144 keys and N(0,1) scores so many rows are sharp that the one
 // recomputing warp sets the pace (B2 H16 T8192 D128: 389 us at W = 48 and 231 at W = 64,
-// against 105 and 104 with hi + lo P), while from 160 keys on hi + lo P costs more than it
-// saves (W = 256: 128 against 115 us).
-constexpr int kPPPreciseWindow = 128;
+// against 105 and 104 with hi + lo P; 138 against 104 at W = 129, whose bands still span
+// two key tiles), while from 152 keys on hi + lo P costs more than it saves (W = 152: 134.5
+// against 125.6 us; W = 256: 128 against 115).
+constexpr int kPPPreciseWindow = 144;
 constexpr uint64_t kPPDrainLimitNs = 200000000ull;
 // Bands of at most this many keys use two MMA issuers (one per query tile), longer ones one.
 constexpr int kPPTwoIssuerWindow = 1024;

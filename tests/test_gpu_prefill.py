@@ -54,8 +54,9 @@ BF16_SHAPES = [
     (2, 2, 333, 128, 8), (1, 3, 95, 64, 5), (1, 2, 33, 128, 4), (1, 1, 7, 128, 8),
     (2, 1, 500, 64, 7), (1, 2, 64, 128, 6), (1, 2, 300, 128, 9), (1, 1, 31, 64, 8),
     (1, 2, 200, 64, 7),
-    # either side of the band length (128 keys) up to which every tile carries P as hi + lo
-    (1, 2, 700, 128, 33), (1, 2, 600, 64, 48), (2, 1, 900, 128, 64), (1, 2, 500, 128, 160),
+    # either side of the band length (144 keys) up to which every tile carries P as hi + lo
+    (1, 2, 700, 128, 33), (1, 2, 600, 64, 48), (2, 1, 900, 128, 64), (1, 2, 500, 128, 129),
+    (1, 2, 600, 128, 144), (1, 2, 500, 64, 145), (1, 2, 500, 128, 160),
 ]
 
 
