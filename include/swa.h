@@ -431,7 +431,8 @@ int swa_decode_split_plan(int64_t B, int64_t H, int64_t D, int64_t W,
  *     one SM's work, then ADAPTIVE for every later launch on that device (see
  *     swa_prefill_auto_state). Results are within the bound either way, but not bitwise the
  *     same across the switch.
- * The modes are process-wide settings read at each launch.
+ * The modes are process-wide settings read at each launch; a CUDA graph that captured a
+ * prefill keeps the kernel chosen when it was captured.
  */
 #define SWA_PREFILL_AUTO 0
 #define SWA_PREFILL_ADAPTIVE 1
