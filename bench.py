@@ -10,8 +10,10 @@ with L2 flushed between steps under "small"; swa_decode over the streaming workl
 streams, H=32, D=128, W=4096 ring, positions uniform in [0, 100000)) under "decode"; the
 chunked streaming prefill (the same streams each taking 128 new tokens,
 swa_chunk_forward) under "chunk"; the multi-head module (cuBLASLt projections around the
-attention, B1 T16384 d_model 4096, 32 heads, W4096) under "module"; and the backward of
-the Mistral-shaped prefill under "backward". Useful prefill FLOPs count the band only:
+attention, B1 T16384 d_model 4096, 32 heads, W4096) under "module"; the backward of
+the Mistral-shaped prefill under "backward"; and the prefill on inputs whose rows a few
+keys dominate (falling scores, B1 H8 T16384 D128 W4096) with adaptive P under "peaked".
+Useful prefill FLOPs count the band only:
 4*B*H*D*sum_i min(i+1, W). Decode bytes are the K/V slots read plus q, out and pos;
 chunk bytes are the ring slots the chunk needs, its q, k, v, out, the appended rows and
 pos.
@@ -353,6 +355,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-peaked", action="store_true",
+                    help="skip the prefill on inputs whose rows a few keys dominate (adaptive P)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--no-module", action="store_true")
@@ -553,6 +557,39 @@ def main():
             "clocks": dclk.summary(), "gpu_launches": args.steps,
         }
 
+    # ------------------------------------------------------------ peaked inputs, adaptive P
+    # Rows that a few keys dominate (falling scores: the oldest key of each band) make the
+    # fast prefill recompute nearly every row; the default mode switches a device to
+    # adaptive P after such a launch. Timed here in the adaptive mode directly.
+    peaked_line = None
+    if not args.no_peaked:
+        torch.cuda.empty_cache()
+        PB, PH, PT, PD, PW, pseed = 1, 8, 16384, 128, 4096, 77
+        pq, pk, pv = (t.to(device) for t in inputs.peaked_prefill_inputs(PB, PH, PT, PD, pseed, "falling"))
+        pout = torch.empty_like(pq)
+        prev_mode = swa.set_prefill_mode(swa.PREFILL_ADAPTIVE)
+        try:
+            pstep = lambda: swa.forward(pq, pk, pv, PW, out=pout)
+            for _ in range(args.warmup):
+                pstep()
+            swa.device_status()
+            psteps = max(3, min(args.steps, 20))
+            with ClockSampler(dev_index) as pclk:
+                pms = timed(pstep, psteps, stream, pg, device) / psteps
+            swa.device_status()
+        finally:
+            swa.set_prefill_mode(prev_mode)
+        pF = band_flops(PB, PH, PT, PD, PW)
+        peaked_line = {
+            "metric": "prefill TFLOP/s, rows dominated by a few keys, adaptive P", "unit": "TFLOP/s",
+            "value": world * pF / (pms * 1e-3) / 1e12, "ms_per_step": pms, "steps": psteps,
+            "config": {"workload": f"falling scores B{PB} H{PH} T{PT} D{PD} W{PW}", "seed": pseed,
+                       "inputs": "q all ones, k_t = -0.05 t + N(0, 0.01^2), v ~ N(0,1), bf16",
+                       "mode": "adaptive"},
+            "clocks": pclk.summary(), "gpu_launches": psteps,
+        }
+        del pq, pk, pv, pout
+
     # ------------------------------------------------------------ chunked streaming prefill
     chunk_line = None
     if not args.no_chunk:
@@ -696,6 +733,7 @@ def main():
         "chunk": chunk_line,
         "module": module_line,
         "backward": backward_line,
+        "peaked": peaked_line,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

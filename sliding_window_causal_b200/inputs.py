@@ -91,6 +91,29 @@ def prefill_inputs(B, H, T, D, dtype, seed):
     return q, k, v
 
 
+def peaked_prefill_inputs(B, H, T, D, seed, kind):
+    """bf16 q, k, v of shape [B,H,T,D] on the CPU whose rows a few keys dominate: q is all
+    ones and every key row is a base value (the same in each of its D elements) plus
+    N(0, 0.01^2) noise. "growing": base 0.05*t, so the newest keys of each band dominate;
+    "falling": -0.05*t, so the oldest do; "spikes": T // 50 keys at random positions get
+    base 1, the rest 0. v ~ N(0, 1)."""
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.ones(B, H, T, D)
+    t = torch.arange(T, dtype=torch.float32)
+    if kind == "growing":
+        base = 0.05 * t
+    elif kind == "falling":
+        base = -0.05 * t
+    elif kind == "spikes":
+        base = torch.zeros(T)
+        base[torch.randint(0, T, (T // 50,), generator=gen)] = 1.0
+    else:
+        raise ValueError(f"unknown kind {kind!r}")
+    k = base[None, None, :, None].expand(B, H, T, D).clone() + 0.01 * torch.randn(B, H, T, D, generator=gen)
+    v = torch.randn(B, H, T, D, generator=gen)
+    return tuple(x.to(torch.bfloat16) for x in (q, k, v))
+
+
 def decode_inputs(B, H, D, W, pos_max, dtype, seed):
     """q [B,H,D], kring and vring [B,H,W,D] i.i.d. N(0,1) rounded to dtype, and
     pos [B] int64 uniform in [0, pos_max), all on the CPU."""

@@ -39,16 +39,5 @@ def sharp_inputs(B, H, T, D, seed, kind):
     """Inputs whose rows are dominated by a few keys: "growing" (scores rise along the
     sequence, so the newest keys dominate), "falling" (they fall, so the oldest keys of
     each band dominate) or "spikes" (a few keys with large scores anywhere). v ~ N(0,1)."""
-    gen = torch.Generator().manual_seed(seed)
-    q = torch.ones(B, H, T, D)
-    t = torch.arange(T, dtype=torch.float32)
-    if kind == "growing":
-        base = 0.05 * t
-    elif kind == "falling":
-        base = -0.05 * t
-    else:
-        base = torch.zeros(T)
-        base[torch.randint(0, T, (T // 50,), generator=gen)] = 1.0
-    k = base[None, None, :, None].expand(B, H, T, D).clone() + 0.01 * torch.randn(B, H, T, D, generator=gen)
-    v = torch.randn(B, H, T, D, generator=gen)
-    return tuple(x.to(torch.bfloat16) for x in (q, k, v))
+    from sliding_window_causal_b200 import inputs
+    return inputs.peaked_prefill_inputs(B, H, T, D, seed, kind)
