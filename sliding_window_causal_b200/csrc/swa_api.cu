@@ -675,7 +675,7 @@ int swa_band_weights(const void* q, const void* k, float* weights, int64_t B, in
     const size_t esz = dtype == SWA_BF16 ? 2 : 4;
     if (!aligned(q, esz) || !aligned(k, esz) || !aligned(weights, 4))
         return fail(SWA_ERR_MISALIGNED, "%s: tensors must be aligned to their element size", fn);
-    int64_t st[2][3];
+    int64_t st[2][3] = {};
     if (int rc = read_strides(fn, strides, 2, B, H, T, D, st)) return rc;
     const int64_t nrows = B * H * T;
     const int64_t blocks = (nrows + swa::kWeightWarps - 1) / swa::kWeightWarps;
