@@ -27,7 +27,9 @@ from ._native import SWA_BF16, SWA_F32, SwaError, check
 
 __all__ = ["forward", "forward_lse", "backward", "band_weights", "decode", "chunk_forward", "ring_append", "mha_forward",
            "mha_workspace_bytes", "forward_host", "device_status", "tile_class", "valid_slots",
-           "split_plan", "set_wait_limit_ns", "timeout_probe", "SwaError"]
+           "split_plan", "set_wait_limit_ns", "timeout_probe", "work_item", "backward_cta_tile",
+           "set_prefill_mode", "prefill_auto_state", "PREFILL_AUTO", "PREFILL_ADAPTIVE", "PREFILL_FAST",
+           "SwaError"]
 
 
 def _torch():
