@@ -88,6 +88,22 @@ def test_backward_deterministic():
     assert all(torch.equal(x, y) for x, y in zip(a, b))
 
 
+def test_backward_outputs_complete_for_the_next_work_on_the_stream():
+    """The query-tile kernel starts while the key-tile kernel's last CTAs run (a
+    programmatic dependent launch) and waits for it before it ends: work enqueued on the
+    stream right after the backward must see all three gradients complete. Sums taken on
+    the stream with no synchronize in between equal the sums taken after one."""
+    q, k, v = (t.to(DEV) for t in inputs.prefill_inputs(1, 16, 4096, 128, torch.bfloat16, 808))
+    do = inputs.prefill_inputs(1, 16, 4096, 128, torch.bfloat16, 809)[0].to(DEV)
+    out, lse = swa.forward_lse(q, k, v, 1024)
+    for _ in range(3):
+        dq, dk, dv = swa.backward(q, k, v, do, 1024, out=out, lse=lse)
+        early = torch.stack([g.float().sum() for g in (dq, dk, dv)])  # same stream, no sync
+        swa.device_status()
+        late = torch.stack([g.float().sum() for g in (dq, dk, dv)])
+        assert torch.equal(early, late)
+
+
 @pytest.mark.parametrize("D,W", [(64, 50), (128, 6)])
 def test_lse_matches_oracle_weights(D, W):
     """forward_lse's lse is log of the sum of exp(scaled score) over each band (W = 6:
